@@ -1,0 +1,183 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a B200 (sm_100a) fused MoE expert layer.
+ *
+ * The layer is the one the source pages describe: a router picks k experts per token,
+ * tokens are dispatched to their experts, each expert applies linear-1 (gate and up
+ * projections), SwiGLU and linear-2, and the expert outputs are combined with the gate
+ * weights (jiqizhixin, "DeepSeek悄悄更新：Mega MoE、FP4 Indexer来了", section
+ * "Mega MoE 是什么？", the paragraph on the conventional dispatch -> linear -> SwiGLU ->
+ * linear -> combine pipeline and the paragraph on fusing it into one mega-kernel).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library allocates no
+ *     memory.  Row-major, contiguous, 16-byte aligned (E2M1 weights: 32-byte aligned).
+ *   - Work is enqueued asynchronously on `stream`; a call returns once its launches are
+ *     enqueued.  Argument errors are returned synchronously, before anything is launched.
+ *   - A failed launch returns MOE_ERR_CUDA.  A device-side failure (a bounded wait that
+ *     gave up) is recorded in a per-device error word read by moe_get_device_error().
+ *   - Shapes: T tokens, H hidden, E experts, k experts per token, I expert intermediate
+ *     size, S = T*k dispatch slots.  Preconditions: T >= 1, 1 <= k <= min(E, 32),
+ *     E <= 1024, H % 128 == 0, I % 128 == 0.
+ *   - Tensor formats (moe_dtype):
+ *       MOE_F32   IEEE binary32
+ *       MOE_BF16  bfloat16
+ *       MOE_E4M3  OCP FP8 E4M3 codes, one byte each; activations carry one fp32
+ *                 power-of-two scale per 1x128 block along the row, weights one fp32
+ *                 power-of-two scale per 128x128 block
+ *       MOE_E2M1  OCP MX FP4 codes, two per byte (element 2i in the low nibble), weights
+ *                 only, one UE8M0 scale byte (value 2^(b-127)) per 1x32 block along K
+ *   - Supported (activation, weight) pairs: (F32, F32), (BF16, BF16), (E4M3, E4M3),
+ *     (E4M3, E2M1).  h (the SwiGLU output) is stored in the activation format (E4M3 with a
+ *     power-of-two scale per 1x128 block); y and out are BF16, except F32 for the F32 layer.
+ */
+#ifndef MOE_H_
+#define MOE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = -1, /* null pointer, bad shape or bad enum value */
+  MOE_ERR_UNSUPPORTED = -2, /* valid but unsupported combination (dtype pair, E > 1024 ...) */
+  MOE_ERR_MISALIGNED = -3,  /* a pointer misses its alignment requirement */
+  MOE_ERR_WORKSPACE = -4,   /* workspace null, too small or not 256-byte aligned */
+  MOE_ERR_CUDA = -5,        /* a CUDA runtime / driver call or a launch failed */
+  MOE_ERR_TIMEOUT = -6,     /* device side: a bounded wait gave up (see moe_get_device_error) */
+  MOE_ERR_DEVICE = -7       /* device side: any other recorded failure */
+} moe_status;
+
+typedef enum moe_dtype { MOE_F32 = 0, MOE_BF16 = 1, MOE_E4M3 = 2, MOE_E2M1 = 3 } moe_dtype;
+
+typedef enum moe_score { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 } moe_score;
+
+/* Workspace queries name the entry point they size. */
+typedef enum moe_op {
+  MOE_OP_DISPATCH = 1,
+  MOE_OP_LINEAR1 = 2,
+  MOE_OP_LINEAR2 = 3,
+  MOE_OP_FUSED_FFN = 4,
+  MOE_OP_FORWARD = 5
+} moe_op;
+
+/* Expert weights.  W1 [E, 2I, H]: rows [0, I) are the gate projection, rows [I, 2I) the up
+ * projection.  W2 [E, H, I].  Both K-major (each output row contiguous over the reduction
+ * dimension).  Scales: E4M3 -> fp32 [E, 2I/128, H/128] and [E, H/128, I/128];
+ * E2M1 -> UE8M0 bytes [E, 2I, H/32] and [E, H, I/32]; F32 / BF16 -> NULL. */
+typedef struct moe_weights {
+  int act; /* moe_dtype of x, x_perm and h */
+  int wt;  /* moe_dtype of W1 and W2 */
+  const void* w1;
+  const void* w1_scales;
+  const void* w2;
+  const void* w2_scales;
+} moe_weights;
+
+/* Router: per token, select k experts and their gate weights.
+ * (youleyou, "DeepSeek 模型更新解读 Tile Kernels 与 DeepEP V2 新特性", section
+ *  "Tile Kernels：逼近硬件极限的底层优化", gating item: top-k expert selection with scoring;
+ *  routing item: weight normalisation.)
+ *   logits   fp32 [T, E], finite (not checked on the device)
+ *   bias     fp32 [E] or NULL; only MOE_SCORE_SIGMOID uses it, for selection only
+ *   score    MOE_SCORE_SOFTMAX: select on the logits; gates = softmax over the selected k
+ *                               (renorm) or the full softmax of the selected (no renorm).
+ *            MOE_SCORE_SIGMOID: s = sigmoid(logit) evaluated as a fixed sequence of
+ *                               correctly rounded fp32 operations; select on s + bias;
+ *                               gates = s / sum(selected s) (renorm) or s.
+ *   topk_idx int32 [T, k] out, experts in rank order (key descending, ties -> lower id)
+ *   topk_w   fp32 [T, k] out, the gates in the same order */
+moe_status moe_route(const float* logits, const float* bias, int T, int E, int k, int score,
+                     int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t stream);
+
+/* Dispatch: permute token rows to experts (stable counting sort by expert).
+ * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: tokens are dispatched to the
+ *  experts; youleyou, routing item: token-to-expert mapping with fused expand.)
+ *   x              [T, H] in format `act` (F32, BF16 or E4M3)
+ *   x_scales       fp32 [T, H/128] for E4M3, else NULL
+ *   topk_idx       int32 [T, k] from moe_route (each expert at most once per token)
+ *   x_perm         [S, H] out: slot p holds the row of token perm_src[p] / k
+ *   x_perm_scales  fp32 [S, H/128] out for E4M3, else NULL
+ *   expert_offsets int32 [E+1] out: slots of expert e are [offsets[e], offsets[e+1]),
+ *                  in ascending token order
+ *   perm_src       int32 [S] out: slot -> t*k + j
+ *   slot_of        int32 [S] out: t*k + j -> slot
+ *   ws             workspace of moe_workspace_size(MOE_OP_DISPATCH, ...) bytes, 256-byte
+ *                  aligned, contents need no initialisation */
+moe_status moe_dispatch(const void* x, const float* x_scales, int act, int T, int H, int E, int k,
+                        const int32_t* topk_idx, void* x_perm, float* x_perm_scales,
+                        int32_t* expert_offsets, int32_t* perm_src, int32_t* slot_of, void* ws,
+                        size_t ws_bytes, cudaStream_t stream);
+
+/* Expert linear-1 + SwiGLU (+ requantisation): for every slot p of expert e,
+ *   gate = x_perm[p] . W1[e, 0:I]^T, up = x_perm[p] . W1[e, I:2I]^T (fp32 accumulation),
+ *   h[p] = silu(gate) * up stored in format W->act; for E4M3 each 1x128 block of h gets the
+ *   scale 2^n with n the smallest integer such that amax <= 448 * 2^n, and codes are
+ *   round-to-nearest-even, saturating.
+ * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: linear layer then SwiGLU;
+ *  FP8 x FP4 paragraph; youleyou, quantisation item: FP8/FP4 quantisation fused with SwiGLU.)
+ *   h        [S, I] out;  h_scales fp32 [S, I/128] out for E4M3, else NULL
+ *   ws       may be NULL (this entry needs no workspace) */
+moe_status moe_expert_linear1(const void* x_perm, const float* x_perm_scales,
+                              const int32_t* expert_offsets, int S, int H, int I, int E,
+                              const moe_weights* W, void* h, float* h_scales, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
+
+/* Expert linear-2: y[p] = h[p] . W2[e]^T for every slot p of expert e, fp32 accumulation,
+ * stored BF16 (F32 for the F32 layer), unweighted.
+ * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: the second linear layer.)
+ *   h [S, I] (+ h_scales fp32 [S, I/128] for E4M3);  y [S, H] out;  ws may be NULL. */
+moe_status moe_expert_linear2(const void* h, const float* h_scales, const int32_t* expert_offsets,
+                              int S, int H, int I, int E, const moe_weights* W, void* y, void* ws,
+                              size_t ws_bytes, cudaStream_t stream);
+
+/* linear-1 + SwiGLU + linear-2 with h kept in the workspace
+ * (moe_workspace_size(MOE_OP_FUSED_FFN, ...) bytes). */
+moe_status moe_fused_ffn(const void* x_perm, const float* x_perm_scales,
+                         const int32_t* expert_offsets, int S, int H, int I, int E,
+                         const moe_weights* W, void* y, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
+/* Combine: out[t] = sum_{j<k} topk_w[t, j] * y[slot_of[t*k + j]], accumulated in fp32 in
+ * rank order j, no atomics (the result is deterministic), stored in out_dt.
+ * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: results are put back
+ *  together; youleyou, routing item: fused reduce.)
+ *   y [S, H] in y_dt (BF16 or F32);  out [T, H] in out_dt (BF16 or F32). */
+moe_status moe_combine(const void* y, int y_dt, const int32_t* slot_of, const float* topk_w,
+                       int T, int k, int H, void* out, int out_dt, cudaStream_t stream);
+
+/* The whole layer: route -> dispatch -> linear-1 + SwiGLU -> linear-2 -> combine, all
+ * intermediates in the workspace (moe_workspace_size(MOE_OP_FORWARD, ...) bytes).
+ * (jiqizhixin, section "Mega MoE 是什么？", the mega-kernel paragraph.)
+ * topk_idx / topk_w / expert_offsets may be NULL; when given, the routing result and the
+ * per-expert offsets are written there too. */
+moe_status moe_forward(const void* x, const float* x_scales, const float* logits,
+                       const float* bias, int score, int renorm, int T, int H, int E, int k,
+                       int I, const moe_weights* W, void* out, int32_t* topk_idx,
+                       float* topk_w, int32_t* expert_offsets, void* ws, size_t ws_bytes,
+                       cudaStream_t stream);
+
+/* Bytes of workspace entry point `op` needs for these shapes (0 for an invalid query). */
+size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, int wt);
+
+/* Synchronises `stream`, then reads and clears the calling device's error word.
+ * Returns MOE_OK, or the recorded MOE_ERR_TIMEOUT / MOE_ERR_DEVICE with *site (may be NULL)
+ * set to the code location that recorded it, or MOE_ERR_CUDA if the synchronisation
+ * itself failed. */
+moe_status moe_get_device_error(cudaStream_t stream, int* site);
+
+/* Static string naming a status code. */
+const char* moe_status_string(int status);
+
+/* Number of this library's kernel launches made by the calling thread since it was
+ * loaded (host-side counter, for accounting in benchmarks). */
+uint64_t moe_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H_ */

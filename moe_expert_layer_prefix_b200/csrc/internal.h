@@ -1,0 +1,56 @@
+// Host-side launchers shared between the library's translation units.  Each returns the
+// cudaError_t of its launch(es); argument checking happens in api.cu before any of these
+// is called.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+void count_launch(int n = 1);
+
+// Dispatch workspace layout: per-chunk counts / bases [C][E] int32 and expert totals [E].
+constexpr int kChunkTokens = 32;
+inline size_t dispatch_ws_bytes(int T, int E) {
+  size_t C = (static_cast<size_t>(T) + kChunkTokens - 1) / kChunkTokens;
+  return ((C * E * 4 + 255) / 256) * 256 + ((static_cast<size_t>(E) * 4 + 255) / 256) * 256;
+}
+
+cudaError_t launch_route(const float* logits, const float* bias, int T, int E, int k, int score,
+                         int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s);
+
+cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes, int T, int H,
+                            int E, int k, const int32_t* topk_idx, void* x_perm,
+                            float* x_perm_scales, int32_t* offsets, int32_t* perm_src,
+                            int32_t* slot_of, void* ws, cudaStream_t s);
+
+cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, const float* topk_w,
+                           int T, int k, int H, void* out, int out_f32, cudaStream_t s);
+
+struct FfnArgs {
+  int act, wt;                 // moe_dtype
+  const void* a;               // x_perm (linear-1) or h (linear-2)
+  const float* a_scales;       // fp32 [S, K/128] or null
+  const int32_t* offsets;      // [E+1]
+  int S, H, I, E;
+  const void* w;               // W1 or W2
+  const void* w_scales;
+  void* out;                   // h (linear-1) or y (linear-2)
+  float* out_scales;           // h_scales (linear-1, E4M3) or null
+  int* err;                    // device error word
+};
+
+cudaError_t launch_linear1_simt(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_linear2_simt(const FfnArgs& a, cudaStream_t s);
+
+// tcgen05 path; returns cudaErrorNotSupported for dtype pairs it does not cover.
+cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s);
+
+int* device_error_word();   // device address of the calling device's error word
+int num_sms();
+
+}  // namespace moe

@@ -1,0 +1,49 @@
+"""Host-only checks of the C ABI: the library loads without a GPU, exports every entry point
+include/moe.h declares, sizes workspaces and names statuses (no kernel is launched)."""
+import os
+import re
+
+import moe_expert_layer_prefix_b200 as M
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", f)).read()
+            names |= set(re.findall(r"^\s*(?:moe_status|size_t|const char\*|uint64_t)\s+(moe_\w+)\(",
+                                    src, re.M))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared()
+    assert {"moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
+            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
+            "moe_get_device_error", "moe_status_string"} <= declared
+    for n in declared:
+        assert hasattr(M._lib, n), n
+    assert set(M.EXPORTS) == declared
+
+
+def test_status_strings():
+    for code, name in M.STATUS.items():
+        assert M.moe_status_string(code) == name
+    assert M.moe_status_string(12345) == "MOE_ERR_UNKNOWN"
+
+
+def test_workspace_sizes():
+    T, H, E, k, I = 8192, 7168, 256, 8, 2048
+    S = T * k
+    assert M.moe_workspace_size("linear1", T, H, E, k, I, "e4m3", "e4m3") == 0
+    ffn = M.moe_workspace_size("fused_ffn", S, H, E, 1, I, "e4m3", "e4m3")
+    assert ffn >= S * I + S * (I // 128) * 4
+    fwd = M.moe_workspace_size("forward", T, H, E, k, I, "e4m3", "e4m3")
+    assert fwd >= S * H + S * I + 2 * S * H     # x_perm + h + y (BF16)
+    assert M.moe_workspace_size("dispatch", T, H, E, k, I, "e4m3", "e4m3") >= (T // 32) * E * 4
+    # invalid queries size to zero
+    assert M.moe_workspace_size("forward", T, H, E, k, I, "bf16", "e4m3") == 0
+    assert M.moe_workspace_size(99, T, H, E, k, I, "e4m3", "e4m3") == 0
+    assert M.moe_workspace_size("forward", 0, H, E, k, I, "e4m3", "e4m3") == 0

@@ -1,0 +1,268 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle.
+
+Integer results (routing indices, counts, offsets, permutations, dispatched bytes) must match
+bit for bit.  Floating-point outputs must satisfy max|gpu - oracle| / rms(oracle) <= 1e-4
+(fp32 layer), 1e-2 (BF16) or 3e-2 (FP8 / FP4).  Sizes are chosen so that the oracle finishes
+in seconds while the GEMMs still span several tiles with ragged tails; the full-size
+workloads are checked on sampled tokens."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests.util import TOL, assert_parity, host_values, oracle_layer, parity_err, weights_of
+
+pytestmark = pytest.mark.gpu
+
+M = pytest.importorskip("moe_expert_layer_prefix_b200")
+DEV = "cuda"
+
+SMALL = {
+    "tiny_f32": synth.WORKLOADS["tiny_f32"],
+    "mixtral_bf16": synth.WORKLOADS["mixtral_bf16"].scaled(T=200, H=512, I=1024),
+    "mixtral_bf16_h384": synth.WORKLOADS["mixtral_bf16"].scaled(T=77, H=384, E=5, I=256),
+    "v3_fp8": synth.WORKLOADS["v3_fp8"].scaled(T=300, H=1024, E=16, k=4, I=512),
+    "decode_fp8_fp4": synth.WORKLOADS["decode_fp8_fp4"].scaled(T=33, H=1024, E=64, I=256),
+    "skewed_fp8_fp4": synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=260, H=512, E=128, I=256),
+}
+
+
+def _inputs(wl):
+    return synth.make_inputs(wl, DEV)
+
+
+# ------------------------------------------------------------------------------- route
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_route_full_size_bit_exact(name):
+    wl = synth.WORKLOADS[name]
+    a = synth.make_activations(wl, DEV)
+    idx, w = M.moe_route(a["logits"], wl.k, wl.score, bias=a["bias"], renorm=wl.renorm)
+    ridx, rw = oracle.route(a["logits"].cpu().numpy(),
+                            None if a["bias"] is None else a["bias"].cpu().numpy(), wl.k,
+                            wl.score, wl.renorm)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    assert np.max(np.abs(w.cpu().numpy() - rw) / rw) < 1e-6
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+@pytest.mark.parametrize("T,E,k", [(1, 8, 1), (5, 8, 8), (37, 1024, 32), (64, 33, 3), (9, 1, 1)])
+def test_route_edges(score, T, E, k):
+    g = torch.Generator(device=DEV).manual_seed(T * 131 + E)
+    logits = torch.randn((T, E), generator=g, device=DEV)
+    logits[0] = 0.5                                         # all tied
+    bias = torch.randn(E, generator=g, device=DEV) * 0.1 if score == "sigmoid" else None
+    for renorm in (True, False):
+        idx, w = M.moe_route(logits, k, score, bias=bias, renorm=renorm)
+        ridx, rw = oracle.route(logits.cpu().numpy(),
+                                None if bias is None else bias.cpu().numpy(), k, score, renorm)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert np.max(np.abs(w.cpu().numpy() - rw) / np.maximum(rw, 1e-30)) < 2e-6
+
+
+# ------------------------------------------------------------------------------- dispatch
+def _check_dispatch(wl, d, idx):
+    r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+    counts, offs, perm_src, slot_of = oracle.dispatch(idx.cpu().numpy(), wl.E)
+    assert np.array_equal(r["expert_offsets"].cpu().numpy(), offs)
+    assert np.array_equal(r["perm_src"].cpu().numpy(), perm_src)
+    assert np.array_equal(r["slot_of"].cpu().numpy(), slot_of)
+    tok = torch.from_numpy(perm_src // wl.k).long().to(DEV)
+    assert torch.equal(r["x_perm"], d["x"][tok])
+    if wl.act == "e4m3":
+        assert torch.equal(r["x_perm_scales"], d["x_scales"][tok])
+    return r
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_dispatch_bit_exact(name):
+    wl = SMALL[name]
+    d = _inputs(wl)
+    idx, _ = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+    _check_dispatch(wl, d, idx)
+
+
+@pytest.mark.parametrize("case", ["one_expert", "empty_experts", "T1"])
+def test_dispatch_edges(case):
+    wl = synth.WORKLOADS["v3_fp8"].scaled(T=70, H=256, E=40, k=3, I=128)
+    if case == "T1":
+        wl = wl.scaled(T=1)
+    d = _inputs(wl)
+    if case == "one_expert":
+        idx = torch.tensor([[7, 3, 9]] * wl.T, dtype=torch.int32, device=DEV)
+    elif case == "empty_experts":
+        idx = torch.stack([torch.randperm(5, device=DEV)[:3] for _ in range(wl.T)]).int() + 30
+    else:
+        idx = torch.tensor([[39, 0, 12]], dtype=torch.int32, device=DEV)
+    _check_dispatch(wl, d, idx)
+
+
+def test_dispatch_full_size_bit_exact():
+    wl = synth.WORKLOADS["skewed_fp8_fp4"]
+    a = synth.make_activations(wl, DEV)
+    idx, _ = M.moe_route(a["logits"], wl.k, wl.score)
+    _check_dispatch(wl, a, idx)
+
+
+# ------------------------------------------------------------------------------- combine
+@pytest.mark.parametrize("ydt", ["bf16", "f32"])
+def test_combine(ydt):
+    T, k, H, E = 123, 5, 768, 20
+    g = torch.Generator(device=DEV).manual_seed(5)
+    logits = torch.randn((T, E), generator=g, device=DEV)
+    idx, w = M.moe_route(logits, k)
+    d = M.moe_dispatch(torch.randn((T, H), device=DEV), idx, E, "f32")
+    y = torch.randn((T * k, H), generator=g, device=DEV)
+    y = y if ydt == "f32" else y.to(torch.bfloat16)
+    out = M.moe_combine(y, d["slot_of"], w)
+    ref = oracle.combine(host_values(y, None, ydt), d["slot_of"].cpu().numpy(),
+                         w.cpu().numpy(), ydt)
+    got = host_values(out, None, ydt)
+    assert_parity(got, ref, ydt, 1e-6 if ydt == "f32" else 1e-3)
+
+
+def test_combine_inverts_dispatch():
+    T, k, H, E = 50, 3, 256, 9
+    x = torch.randn((T, H), device=DEV).to(torch.bfloat16)
+    idx, _ = M.moe_route(torch.randn((T, E), device=DEV), k)
+    d = M.moe_dispatch(x, idx, E, "bf16")
+    w = torch.zeros((T, k), device=DEV)
+    w[:, 0] = 1.0
+    assert torch.equal(M.moe_combine(d["x_perm"], d["slot_of"], w), x)
+
+
+# ------------------------------------------------------------------------------- expert FFN
+def _expert_ffn_ref(L, wl, xh_rows_by_expert, offsets):
+    """oracle y and stored h, expert by expert, on given dequantised input rows."""
+    S = offsets[-1]
+    y = np.zeros((S, wl.H))
+    h = np.zeros((S, wl.I))
+    for e in range(wl.E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        if a == b:
+            continue
+        w1, w2 = L.expert_weights(e)
+        y[a:b], h[a:b] = oracle.expert_ffn(xh_rows_by_expert[a:b], w1, w2, wl.act,
+                                           return_h=True)
+    return y, h
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_linear1_linear2(name):
+    wl = SMALL[name]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    idx, _ = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+    r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+    h, hs = M.moe_expert_linear1(r["x_perm"], r["expert_offsets"], W,
+                                 x_perm_scales=r["x_perm_scales"])
+    y = M.moe_expert_linear2(h, r["expert_offsets"], W, h_scales=hs)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error()[0] == 0
+    L = oracle_layer(wl, d)
+    offs = r["expert_offsets"].cpu().numpy()
+    xp = host_values(r["x_perm"], r["x_perm_scales"], wl.act)
+    yref, href = _expert_ffn_ref(L, wl, xp, offs)
+    hg = host_values(h, hs, wl.act)
+    if wl.act == "e4m3":
+        # h codes: the GPU decides on its fp32 h, the oracle on its fp64 h rounded to fp32,
+        # so a code may land one E4M3 step away (a block scale two-fold away when amax sits
+        # on a power-of-two boundary); everything else must be identical
+        sub = np.repeat(np.maximum(hs.cpu().numpy(), 1e-30).astype(np.float64), 128, 1)
+        dh = np.abs(hg - href)
+        assert np.all((dh <= 0.126 * np.abs(href) + 1e-30) | (dh <= 2 * 2 ** -9 * sub))
+        assert np.mean(hg != href) < 0.01
+    else:
+        assert_parity(hg, href, wl.act, 1e-5)
+    # y: linear-2 alone, on the GPU's own h (only accumulation order and the output
+    # rounding differ)
+    y2ref = np.zeros_like(yref)
+    for e in range(wl.E):
+        a, b = int(offs[e]), int(offs[e + 1])
+        if a < b:
+            _, w2 = L.expert_weights(e)
+            y2ref[a:b] = hg[a:b] @ w2.T
+    yfmt = "f32" if wl.act == "f32" else "bf16"
+    yg = host_values(y, None, yfmt)
+    assert_parity(yg, y2ref, yfmt, 1e-5 if wl.act == "f32" else 1e-3)
+    # y against the oracle's own h
+    assert_parity(yg, yref, yfmt, TOL[wl.act])
+
+
+# ------------------------------------------------------------------------------- forward
+@pytest.mark.parametrize("name", list(SMALL))
+def test_forward_end_to_end(name):
+    wl = SMALL[name]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
+    out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
+                        renorm=wl.renorm, x_scales=d["x_scales"], topk_idx=idx)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error()[0] == 0
+    L = oracle_layer(wl, d)
+    r = oracle.forward(L, return_all=True)
+    assert np.array_equal(idx.cpu().numpy(), r["topk_idx"])
+    fmt = "f32" if wl.act == "f32" else "bf16"
+    assert_parity(host_values(out, None, fmt), r["out"], fmt, TOL[wl.act])
+
+
+def test_forward_equals_unfused_chain():
+    wl = SMALL["v3_fp8"]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
+                        x_scales=d["x_scales"])
+    idx, w = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+    r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+    y = M.moe_fused_ffn(r["x_perm"], r["expert_offsets"], W, x_perm_scales=r["x_perm_scales"])
+    out2 = M.moe_combine(y, r["slot_of"], w)
+    assert torch.equal(out, out2)                  # same kernels, same order: bitwise equal
+
+
+def test_forward_deterministic():
+    wl = SMALL["skewed_fp8_fp4"]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    a = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, x_scales=d["x_scales"])
+    b = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, x_scales=d["x_scales"])
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("name", ["v3_fp8", "decode_fp8_fp4", "mixtral_bf16", "skewed_fp8_fp4"])
+def test_forward_full_size_sampled(name):
+    """The full-size workload in the benchmark's launch configuration; routing is compared
+    for every token, the output on a few sampled tokens."""
+    wl = synth.WORKLOADS[name]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
+    out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
+                        x_scales=d["x_scales"], topk_idx=idx)
+    torch.cuda.synchronize()
+    assert M.moe_get_device_error()[0] == 0
+    L = oracle_layer(wl, d, lazy_weights=True)
+    ridx, _ = oracle.route(L.logits, L.bias, wl.k, wl.score, wl.renorm)
+    assert np.array_equal(idx.cpu().numpy(), ridx)
+    toks = np.random.default_rng(0).choice(wl.T, 3, replace=False)
+    ref = oracle.forward_tokens(L, toks)
+    got = host_values(out[torch.from_numpy(toks).to(DEV)], None, "bf16")
+    # the RMS of a 3-token sample is noisy; normalise by the full output's RMS
+    full_rms = float(out.float().pow(2).mean().sqrt())
+    mx, _ = parity_err(got, ref, "bf16", full_rms)
+    assert mx <= TOL[wl.act]
+
+
+# ------------------------------------------------------------------------------- errors
+def test_invalid_arguments_rejected_before_launch():
+    x = torch.zeros((4, 128), device=DEV)
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_route(torch.zeros((4, 2000), device=DEV), 2)
+    assert ei.value.status == -2
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_route(torch.zeros((4, 8), device=DEV), 9)
+    assert ei.value.status == -2
+    idx = torch.zeros((4, 1), dtype=torch.int32, device=DEV)
+    with pytest.raises(M.MoeError) as ei:
+        M.moe_dispatch(x, idx, 8, "f32", ws=torch.empty(1, dtype=torch.uint8, device=DEV))
+    assert ei.value.status == -4
