@@ -46,6 +46,9 @@ constexpr int kStages = 4;
 constexpr int kATileBytes = kBM * kRowBytes;     // 16 KB
 constexpr int kBTileBytes = kBN * kRowBytes;     // 32 KB
 constexpr int kStageBytes = kATileBytes + kBTileBytes;
+// E2M1 tiles are expanded to one byte per element in shared memory, but the copy's
+// transaction count is the packed size (half a byte per element).
+constexpr int kStageBytesE2M1 = kATileBytes + kBTileBytes / 2;
 constexpr int kSfaBytes = 512;                   // 128 rows x 4 UE8M0
 constexpr int kSfbBytes = 1024;                  // 256 rows x 4 UE8M0
 constexpr int kTmemCols = 512;
@@ -183,7 +186,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         const int brow1 = kSwiGLU ? tile.e * p.w_rows + p.I + tile.nb * 128 : brow0 + 128;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&ss.empty[stage], phase ^ 1u, p.err, SITE_GEMM_EMPTY, abort)) break;
-          mbar_arrive_expect_tx(&ss.full[stage], kStageBytes);
+          mbar_arrive_expect_tx(&ss.full[stage], kBFmt == 5 ? kStageBytesE2M1 : kStageBytes);
           const int kx = kb * kElemsPerRow;
           tma_load_2d(sA + stage * kATileBytes, &tmA, &ss.full[stage], kx, tile.m0);
           tma_load_2d(sB + stage * kBTileBytes, &tmB, &ss.full[stage], kx, brow0);

@@ -28,6 +28,13 @@ SMALL = {
 }
 
 
+@pytest.fixture(autouse=True)
+def _clear_device_error():
+    """Each test starts with a clear device error word (and asserts on its own errors)."""
+    M.moe_get_device_error()
+    yield
+
+
 def _inputs(wl):
     return synth.make_inputs(wl, DEV)
 
@@ -173,7 +180,7 @@ def test_linear1_linear2(name):
         assert np.all((dh <= 0.126 * np.abs(href) + 1e-30) | (dh <= 2 * 2 ** -9 * sub))
         assert np.mean(hg != href) < 0.01
     else:
-        assert_parity(hg, href, wl.act, 1e-5)
+        assert_parity(hg, href, wl.act, 1e-5 if wl.act == "f32" else 2e-3)
     # y: linear-2 alone, on the GPU's own h (only accumulation order and the output
     # rounding differ)
     y2ref = np.zeros_like(yref)
@@ -184,7 +191,7 @@ def test_linear1_linear2(name):
             y2ref[a:b] = hg[a:b] @ w2.T
     yfmt = "f32" if wl.act == "f32" else "bf16"
     yg = host_values(y, None, yfmt)
-    assert_parity(yg, y2ref, yfmt, 1e-5 if wl.act == "f32" else 1e-3)
+    assert_parity(yg, y2ref, yfmt, 1e-5 if wl.act == "f32" else 2e-3)
     # y against the oracle's own h
     assert_parity(yg, yref, yfmt, TOL[wl.act])
 
@@ -226,6 +233,7 @@ def test_forward_deterministic():
     W = weights_of(wl, d)
     a = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, x_scales=d["x_scales"])
     b = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, x_scales=d["x_scales"])
+    assert M.moe_get_device_error()[0] == 0
     assert torch.equal(a, b)
 
 
