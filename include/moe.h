@@ -161,6 +161,26 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
                        float* topk_w, int32_t* expert_offsets, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
 
+/* moe_dispatch without a caller workspace, for callers that cannot allocate device memory
+ * (a host with no device allocator of its own, a runtime that forbids allocations after
+ * start-up, or a path that must not call cudaMalloc / cudaFree because they can synchronise
+ * the device).  The source pages have no counterpart to this entry point; it exists for
+ * those callers only.
+ *   Arguments, outputs and results are those of moe_dispatch, minus ws / ws_bytes.
+ *   Scratch comes from a 4 MiB buffer compiled into the library, held by every device that
+ *   loads it until the process exits.  Shapes whose dispatch workspace exceeds it
+ *   (moe_workspace_size(MOE_OP_DISPATCH, ...) > 4 MiB; e.g. T > 32736 at E = 1024) return
+ *   MOE_ERR_WORKSPACE before anything is launched.
+ *   The first call on each device looks up the buffer's device address (with that device
+ *   current); make that first call before any stream capture.
+ *   All calls on a device share the buffer: nothing needs clearing between calls, but calls
+ *   that may overlap on the GPU (other streams, other host threads) race and must be
+ *   serialised by the caller. */
+moe_status moe_dispatch_noalloc(const void* x, const float* x_scales, int act, int T, int H, int E,
+                                int k, const int32_t* topk_idx, void* x_perm,
+                                float* x_perm_scales, int32_t* expert_offsets, int32_t* perm_src,
+                                int32_t* slot_of, cudaStream_t stream);
+
 /* Bytes of workspace entry point `op` needs for these shapes (0 for an invalid query). */
 size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, int wt);
 

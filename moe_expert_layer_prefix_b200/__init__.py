@@ -6,7 +6,7 @@ Torch provides device memory and the current stream.  The entry points keep the 
 moe_combine, moe_forward, moe_workspace_size, moe_get_device_error, moe_status_string);
 outputs that are not passed in are allocated with torch.empty.
 
-The library must have been built (``python -m moe_expert_layer_prefix_b200.build``);
+The library must have been built (``python moe_expert_layer_prefix_b200/build.py``);
 importing this package without it raises ImportError -- there is no fallback.
 """
 from __future__ import annotations
@@ -20,7 +20,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libmoe.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
-                      "`python -m moe_expert_layer_prefix_b200.build`")
+                      "`python moe_expert_layer_prefix_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 MOE_OK = 0
@@ -33,7 +33,8 @@ OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5}
 
 EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
-           "moe_get_device_error", "moe_status_string", "moe_launch_count")
+           "moe_get_device_error", "moe_status_string", "moe_launch_count",
+           "moe_dispatch_noalloc")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -58,6 +59,8 @@ _linear2 = _sig("moe_expert_linear2", _I, [_P, _P, _P, _I, _I, _I, _I,
                                            ctypes.POINTER(MoeWeights), _P, _P, _Z, _P])
 _fused_ffn = _sig("moe_fused_ffn", _I, [_P, _P, _P, _I, _I, _I, _I, ctypes.POINTER(MoeWeights),
                                         _P, _P, _Z, _P])
+_dispatch_noalloc = _sig("moe_dispatch_noalloc", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
+                                                      _P, _P, _P, _P])
 _combine = _sig("moe_combine", _I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _P])
 _forward = _sig("moe_forward", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                     ctypes.POINTER(MoeWeights), _P, _P, _P, _P, _P, _Z, _P])
@@ -243,4 +246,17 @@ def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=Tru
                     int(renorm), T, H, E, k, W.I, ctypes.byref(W.c), _ptr(out), _ptr(topk_idx),
                     _ptr(topk_w), _ptr(expert_offsets), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
+    return out
+
+
+def moe_dispatch_noalloc(x, topk_idx, E, act, out, x_scales=None, stream=None):
+    """moe_dispatch for callers that cannot allocate device memory: the library's built-in
+    scratch buffer replaces the workspace.  `out` must hold every output tensor (x_perm,
+    x_perm_scales for E4M3, expert_offsets, perm_src, slot_of); nothing is allocated here."""
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    _check(_dispatch_noalloc(_ptr(x), _ptr(x_scales), DTYPES[act], T, H, E, k, _ptr(topk_idx),
+                             _ptr(out["x_perm"]), _ptr(out.get("x_perm_scales")),
+                             _ptr(out["expert_offsets"]), _ptr(out["perm_src"]),
+                             _ptr(out["slot_of"]), _stream(stream)), "moe_dispatch_noalloc")
     return out
