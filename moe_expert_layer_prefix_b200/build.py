@@ -1,6 +1,8 @@
 """Builds libmoe.so in-tree with nvcc for sm_100a (no JIT; shapes are runtime arguments).
 
-    python -m moe_expert_layer_prefix_b200.build [--force]
+    python moe_expert_layer_prefix_b200/build.py [--force]
+
+(Run by path, not with -m: importing the package would load the library being rebuilt.)
 
 Each .cu under csrc/ compiles to an object under _build/ (in parallel), then one shared
 library is linked next to this file.  The CUDA runtime is linked statically and the driver
