@@ -126,6 +126,15 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def workload(args) -> synth.Workload:
+    """The named workload, optionally shrunk (--T/--E) for a profiling capture."""
+    wl = synth.WORKLOADS[args.workload]
+    over = {n: v for n, v in (("T", args.T), ("E", args.E)) if v is not None}
+    if over:
+        wl = wl.scaled(name=wl.name + "_" + "_".join(f"{n}{v}" for n, v in over.items()), **over)
+    return wl
+
+
 def algorithmic(wl: synth.Workload, touched: int):
     """Algorithmic bytes / FLOPs per stage (one launch of each stage per step)."""
     T, H, E, k, I, S = wl.T, wl.H, wl.E, wl.k, wl.I, wl.S
@@ -156,7 +165,8 @@ def algorithmic(wl: synth.Workload, touched: int):
 def run_native(args, ws, rank, local):
     import moe_expert_layer_prefix_b200 as M
 
-    wl = synth.WORKLOADS[args.workload]
+    wl = workload(args)
+    M.moe_set_gemm_tiles(args.tiles)
     dev = torch.device("cuda", torch.cuda.current_device())
     d = synth.make_inputs(wl, dev)
     W = M.Weights(wl.act, wl.wt, d["w1"], d["w2"], d["w1_scales"], d["w2_scales"])
@@ -367,7 +377,7 @@ def cpu_baseline(wl, d, ntok):
 
 def run_reference(args, ws, rank):
     import oracle
-    wl = synth.WORKLOADS[args.workload]
+    wl = workload(args)
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     d = synth.make_inputs(wl, dev)          # input generation only; the oracle runs on host
     L = _oracle_layer(wl, d)
@@ -407,6 +417,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="v3_fp8", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair"],
+                    help="tile shape of the expert GEMMs")
+    ap.add_argument("--T", type=int, default=None, help="override T (profiling captures)")
+    ap.add_argument("--E", type=int, default=None, help="override E (profiling captures)")
     ap.add_argument("--cpu-tokens", type=int, default=3)
     ap.add_argument("--ref-tokens", type=int, default=1)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -193,9 +193,15 @@ moe_status moe_get_device_error(cudaStream_t stream, int* site);
 /* Static string naming a status code. */
 const char* moe_status_string(int status);
 
-/* Number of this library's kernel launches made by the calling thread since it was
- * loaded (host-side counter, for accounting in benchmarks). */
+/* Number of this library's kernel launches made since it was loaded (host-side counter,
+ * for accounting in benchmarks). */
 uint64_t moe_launch_count(void);
+
+/* Process-wide tile shape of the tensor-core expert GEMMs (a tuning and testing knob):
+ * 0 automatic (CTA pairs, M = 256 per tile, when S >= 128 * E; single CTAs, M = 128,
+ * otherwise), 1 always single CTAs, 2 always CTA pairs.  Results are identical up to fp32
+ * accumulation order.  Returns MOE_ERR_INVALID_ARG for any other value. */
+moe_status moe_set_gemm_tiles(int mode);
 
 #ifdef __cplusplus
 }

@@ -34,7 +34,7 @@ OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5}
 EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
            "moe_get_device_error", "moe_status_string", "moe_launch_count",
-           "moe_dispatch_noalloc")
+           "moe_dispatch_noalloc", "moe_set_gemm_tiles")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -68,6 +68,7 @@ _ws_size = _sig("moe_workspace_size", _Z, [_I, _I, _I, _I, _I, _I, _I, _I])
 _get_err = _sig("moe_get_device_error", _I, [_P, ctypes.POINTER(ctypes.c_int)])
 _status_string = _sig("moe_status_string", ctypes.c_char_p, [_I])
 _launch_count = _sig("moe_launch_count", ctypes.c_uint64, [])
+_set_tiles = _sig("moe_set_gemm_tiles", _I, [_I])
 
 
 class MoeError(RuntimeError):
@@ -82,6 +83,15 @@ def moe_status_string(status: int) -> str:
 
 def moe_launch_count() -> int:
     return int(_launch_count())
+
+
+TILES = {"auto": 0, "single": 1, "pair": 2}
+
+
+def moe_set_gemm_tiles(mode="auto"):
+    """Process-wide tile shape of the expert GEMMs: 'auto', 'single' (M = 128 per CTA) or
+    'pair' (M = 256 per 2-CTA cluster)."""
+    _check(_set_tiles(TILES[mode] if isinstance(mode, str) else mode), "moe_set_gemm_tiles")
 
 
 def _ptr(t):

@@ -13,6 +13,7 @@ __device__ int g_error_word[2];
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_tile_mode{0};
 
 constexpr int kMaxDevices = 64;
 int* g_err_ptr[kMaxDevices] = {};
@@ -27,6 +28,8 @@ int current_device() {
 }  // namespace
 
 void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
+
+int gemm_tile_mode() { return g_tile_mode.load(); }
 
 int* device_error_word() {
   const int d = current_device();
@@ -129,6 +132,12 @@ const char* moe_status_string(int status) {
 }
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
+
+moe_status moe_set_gemm_tiles(int mode) {
+  if (mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  g_tile_mode.store(mode);
+  return MOE_OK;
+}
 
 size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, int wt) {
   if (T < 1 || H < 1 || E < 1 || k < 1 || I < 1) return 0;

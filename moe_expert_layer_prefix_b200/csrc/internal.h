@@ -51,6 +51,7 @@ cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s);
 
 int* device_error_word();   // device address of the calling device's error word
+int gemm_tile_mode();       // 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles
 int num_sms();
 
 }  // namespace moe

@@ -25,6 +25,12 @@ SMALL = {
     "v3_fp8": synth.WORKLOADS["v3_fp8"].scaled(T=300, H=1024, E=16, k=4, I=512),
     "decode_fp8_fp4": synth.WORKLOADS["decode_fp8_fp4"].scaled(T=33, H=1024, E=64, I=256),
     "skewed_fp8_fp4": synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=260, H=512, E=128, I=256),
+    # at least 128 rows per expert on average: 2-CTA (M = 256) tiles
+    "v3_fp8_pair": synth.WORKLOADS["v3_fp8"].scaled(T=600, H=1024, E=8, k=4, I=512),
+    "mixtral_bf16_pair": synth.WORKLOADS["mixtral_bf16"].scaled(T=512, H=512, E=4, I=512),
+    "mixtral_bf16_h384_pair": synth.WORKLOADS["mixtral_bf16"].scaled(T=400, H=384, E=3, I=256),
+    "skewed_fp8_fp4_pair": synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=512, H=512, E=32, k=8,
+                                                                    I=256),
 }
 
 
