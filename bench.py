@@ -212,8 +212,15 @@ def run_native(args, ws, rank, local):
         M.moe_combine(y, disp["slot_of"], gw, out=out, stream=stream)
         mark(5)
 
+    fws = M.workspace(M.moe_workspace_size("forward", T, H, E, k, I, wl.act, wl.wt), dev)
+
+    def fused_step():
+        M.moe_forward(d["x"], d["logits"], W, k, wl.score, bias=d["bias"], renorm=wl.renorm,
+                      x_scales=d["x_scales"], out=out, ws=fws, stream=stream)
+
     for _ in range(args.warmup):
         step()
+        fused_step()
     torch.cuda.synchronize()
     st, site = M.moe_get_device_error()
     if st != 0:
@@ -224,22 +231,36 @@ def run_native(args, ws, rank, local):
     clocks = Clocks(local)
     clocks.start()
     time.sleep(0.3)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    # (1) the headline step: moe_forward, one persistent launch per step
     barrier(ws)
     torch.cuda.synchronize()
     n0 = M.moe_launch_count()
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        fused_step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    launches = M.moe_launch_count() - n0
+    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
+    ms = ms_total / args.steps
+    # (2) the same layer as the chain of entry points, CUDA events between the calls
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    barrier(ws)
+    torch.cuda.synchronize()
     t0.record(stream)
     for i in range(args.steps):
         step(evs[i])
     t1.record(stream)
     torch.cuda.synchronize()
     barrier(ws)
-    launches = M.moe_launch_count() - n0
+    chain_ms = max_over_ranks(t0.elapsed_time(t1), ws) / args.steps
     clk = clocks.stop()
-    ms_total = max_over_ranks(t0.elapsed_time(t1), ws)
-    ms = ms_total / args.steps
+    st, site = M.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {M.moe_status_string(st)} at site {site}")
     stage_ms = {n: float(np.mean([evs[i][j].elapsed_time(evs[i][j + 1])
                                   for i in range(args.steps)]))
                 for j, n in enumerate(names)}
@@ -257,7 +278,6 @@ def run_native(args, ws, rank, local):
     x_d = torch.empty_like(d["x"])
     l_d = torch.empty_like(d["logits"])
     xs_d = torch.empty_like(d["x_scales"]) if xs_h is not None else None
-    fws = M.workspace(M.moe_workspace_size("forward", T, H, E, k, I, wl.act, wl.wt), dev)
 
     def e2e_step():
         x_d.copy_(x_h, non_blocking=True)
@@ -325,12 +345,16 @@ def run_native(args, ws, rank, local):
                    "l2": "inputs larger than L2 (expert weights >> 126 MB), no flush",
                    "parallelism": f"replicas x{ws}"},
         "tflops": wl.flops() / (ms / 1e3) / 1e12 * ws,
+        "step": "moe_forward (one persistent launch per step)",
+        "chain_ms_per_step": chain_ms,
         "stage_ms": stage_ms,
         "roofline": roof,
         "e2e": {"value": T * ws / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "path": "moe_forward with pinned host in/out"},
         "gpu_launches": int(launches),
+        "gpu_launches_note": "library kernel launches in the headline timed region (the "
+                             "per-stage breakdown loop adds 8 per step)",
         "clocks": clk,
     }
     if ws == 1 and not args.no_cpu_baseline:

@@ -162,6 +162,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       b += dispatch_ws_bytes(T, E);
       b += h_bytes(S, I, act);
       b += round256(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));  // y
+      b += 256;                                                               // grid barrier
       return b;
     }
     default:
@@ -321,9 +322,54 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
   void* dws = take(dispatch_ws_bytes(T, E));
   void* ffn_ws = take(h_bytes(S, I, act));
   void* y = take(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));
+  uint32_t* bar = reinterpret_cast<uint32_t*>(take(256));
   if (topk_idx_out) topk_idx = topk_idx_out;
   if (topk_w_out) topk_w = topk_w_out;
   if (offsets_out) offsets = offsets_out;
+
+  if (act != MOE_F32) {
+    // tensor-core formats: the whole layer in one persistent launch
+    if (!aligned(logits, 4) || (bias && !aligned(bias, 4)) || !aligned(out, 16) ||
+        !aligned(x, 16) || (x_scales && !aligned(x_scales, 4)))
+      return MOE_ERR_MISALIGNED;
+    if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+    const size_t hsz = round256(static_cast<size_t>(S) * I * act_bytes(act));
+    ForwardArgs fa;
+    fa.x = x;
+    fa.x_scales = act == MOE_E4M3 ? x_scales : nullptr;
+    fa.logits = logits;
+    fa.bias = score == MOE_SCORE_SIGMOID ? bias : nullptr;
+    fa.sigmoid = score == MOE_SCORE_SIGMOID;
+    fa.renorm = renorm != 0;
+    fa.T = T;
+    fa.H = H;
+    fa.E = E;
+    fa.k = k;
+    fa.I = I;
+    fa.act = act;
+    fa.wt = W->wt;
+    fa.w1 = W->w1;
+    fa.w1_scales = W->w1_scales;
+    fa.w2 = W->w2;
+    fa.w2_scales = W->w2_scales;
+    fa.topk_idx = topk_idx;
+    fa.topk_w = topk_w;
+    fa.offsets = offsets;
+    fa.perm_src = perm_src;
+    fa.slot_of = slot_of;
+    fa.x_perm = x_perm;
+    fa.x_perm_scales = x_perm_scales;
+    fa.cnt = static_cast<int32_t*>(dws);
+    fa.totals = reinterpret_cast<int32_t*>(
+        static_cast<char*>(dws) + round256(static_cast<size_t>((T + kChunkTokens - 1) / kChunkTokens) * E * 4));
+    fa.h = ffn_ws;
+    fa.h_scales = act == MOE_E4M3 ? reinterpret_cast<float*>(static_cast<char*>(ffn_ws) + hsz) : nullptr;
+    fa.y = y;
+    fa.out = out;
+    fa.bar = bar;
+    fa.err = device_error_word();
+    return cuda_status(launch_forward_fused(fa, stream));
+  }
 
   st = moe_route(logits, bias, T, E, k, score, renorm, topk_idx, topk_w, stream);
   if (st != MOE_OK) return st;

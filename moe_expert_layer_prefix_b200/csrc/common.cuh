@@ -177,6 +177,11 @@ __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m
       : "memory");
 }
 
+// Orders this thread's generic-proxy global writes before later async-proxy (TMA) reads.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // Orders this thread's generic-proxy shared-memory writes before later async-proxy
 // (TMA / tcgen05) accesses.
 __device__ __forceinline__ void fence_proxy_async_smem() {
@@ -375,6 +380,46 @@ __device__ __forceinline__ int e4m3_scale_exponent(float a) {
 
 __device__ __forceinline__ float exp2i(int n) {  // 2^n for -126 <= n <= 127
   return __uint_as_float(static_cast<uint32_t>(n + 127) << 23);
+}
+
+// ---------------------------------------------------------------------------------------
+// grid-wide barrier for co-resident (cooperative) grids: bar[0] arrivals, bar[1] generation
+// (both zero before the launch).  Bounded: gives up after kWaitLimitCycles, records
+// MOE_ERR_TIMEOUT at SITE_GRID_BARRIER and returns false.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {
+  __syncthreads();
+  __shared__ int ok_s;
+  if (threadIdx.x == 0) {
+    int ok = 1;
+    const uint32_t gen = ld_acquire_gpu(bar + 1);
+    __threadfence();
+    const uint32_t arrived = atomicAdd(bar, 1u);
+    if (arrived == gridDim.x - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      const long long t0 = clock64();
+      while (ld_acquire_gpu(bar + 1) == gen) {
+        if (clock64() - t0 > kWaitLimitCycles) {
+          report_error(err, MOE_ERR_TIMEOUT, SITE_GRID_BARRIER);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
 }
 
 }  // namespace moe

@@ -1,0 +1,232 @@
+// The whole MoE layer in one persistent launch: route -> dispatch -> linear-1 + SwiGLU +
+// requant -> linear-2 -> combine.
+//
+// This is the "mega-kernel" of the source pages: dispatch, both linear layers, SwiGLU and
+// combine fused into one kernel instead of one launch per step (jiqizhixin,
+// "DeepSeek悄悄更新：Mega MoE、FP4 Indexer来了", section "Mega MoE 是什么？", the mega-kernel
+// paragraph; the routing step in front of it follows youleyou, "DeepSeek 模型更新解读 Tile
+// Kernels 与 DeepEP V2 新特性", Tile Kernels feature list, gating item).  On one GPU there is
+// no communication to overlap; what the fusion removes is the launch gaps and the host
+// round trips between the steps.
+//
+// One CTA per SM, all co-resident (cooperative launch).  Phases are separated by grid-wide
+// barriers with bounded waits; each phase runs exactly the device code of the standalone
+// kernels (route.cuh, dispatch.cuh, gemm_tc.cuh, combine.cuh), so moe_forward produces the
+// same bytes as the unfused chain of entry points.  Data produced by one phase is read by the
+// next through L2 (ld.global.cg), and the phases whose output a TMA copy reads (x_perm, h)
+// end with a generic-to-async proxy fence.  The shared memory of the GEMM ring doubles as
+// the dispatch phases' scratch (chunk masks, slot tables, offsets), and one TMEM
+// allocation serves both GEMM phases, whose pipeline counters carry over.
+#include "combine.cuh"
+#include "common.cuh"
+#include "dispatch.cuh"
+#include "gemm_tc.cuh"
+#include "internal.h"
+#include "route.cuh"
+
+namespace moe {
+namespace {
+
+using namespace gemm;
+
+struct FwdParams {
+  const void* x;
+  const float* x_scales;
+  const float* logits;
+  const float* bias;
+  int sigmoid, renorm, T, H, E, k, C;
+  int row_bytes;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* offsets;
+  int32_t* perm_src;
+  int32_t* slot_of;
+  void* x_perm;
+  float* x_perm_scales;
+  int32_t* cnt;
+  int32_t* totals;
+  void* y;
+  void* out;
+  uint32_t* bar;
+  int* err;
+  TcParams l1, l2;
+};
+
+template <bool kBS, int kBFmt, bool kE4>
+__global__ void __launch_bounds__(kThreads, 1)
+moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
+                   const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW2,
+                   const FwdParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const Smem sm = carve<1>(smem_raw);
+  gemm_init<1, kBS>(sm, &tmX, 1);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmW1);
+    tma_prefetch_desc(&tmH);
+    tma_prefetch_desc(&tmW2);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nwarps = kThreads / 32;
+  const int gw = blockIdx.x * nwarps + warp, GW = gridDim.x * nwarps;
+  // dispatch scratch inside the (idle) GEMM ring: per-warp chunk masks in the A stages,
+  // slot tables, scan partials and offsets in the B stages
+  uint32_t* mask = reinterpret_cast<uint32_t*>(sm.sA) + warp * p.E;
+  int32_t(*sslot)[32] = reinterpret_cast<int32_t(*)[32]>(sm.sB) + warp * kChunkTokens;
+  int32_t(*part)[33] = reinterpret_cast<int32_t(*)[33]>(sm.sB + nwarps * kChunkTokens * 32 * 4);
+  int32_t* soffs = reinterpret_cast<int32_t*>(sm.sB + nwarps * kChunkTokens * 32 * 4 + 32 * 33 * 4);
+  int32_t* wsum = soffs + 1028;
+
+  // 1. route: one warp per token
+  for (int t = gw; t < p.T; t += GW)
+    route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+  grid_sync(p.bar, p.err);
+
+  // 2. per-chunk expert counts
+  for (int c = gw; c < p.C; c += GW) hist_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, lane, p.cnt);
+  grid_sync(p.bar, p.err);
+
+  // 3. per-expert scans over the chunks (32 experts per CTA pass)
+  for (int g = blockIdx.x; g < (p.E + 31) / 32; g += gridDim.x)
+    scan_group(p.cnt, p.E, p.C, p.totals, g, nwarps, warp, lane, part);
+  grid_sync(p.bar, p.err);
+
+  // 4. expert offsets (every CTA keeps its own copy; CTA 0 publishes them)
+  offsets_from_totals(p.totals, p.E, soffs, wsum);
+  if (blockIdx.x == 0)
+    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.offsets[e] = soffs[e];
+
+  // 5. slots, permutation and row copies
+  for (int c = gw; c < p.C; c += GW)
+    scatter_chunk(mask, sslot, static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes,
+                  p.H / 128, p.topk_idx, p.T, p.E, p.k, c, p.cnt, soffs,
+                  static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, p.perm_src, p.slot_of, lane);
+  fence_proxy_async_global();  // x_perm is read by TMA next
+  grid_sync(p.bar, p.err);
+
+  // 6. linear-1 + SwiGLU + requantisation
+  Pipe pipe;
+  gemm_prefix<1>(sm, p.offsets, p.E, p.l1.n_tiles);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  gemm_phase<1, kBS, kBFmt, true, kE4>(&tmX, &tmW1, p.l1, sm, pipe);
+  fence_proxy_async_global();  // h is read by TMA next
+  grid_sync(p.bar, p.err);
+
+  // 7. linear-2
+  gemm_prefix<1>(sm, p.offsets, p.E, p.l2.n_tiles);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  gemm_phase<1, kBS, kBFmt, false, false>(&tmH, &tmW2, p.l2, sm, pipe);
+  grid_sync(p.bar, p.err);
+
+  // 8. combine: one warp per token
+  for (int t = gw; t < p.T; t += GW)
+    combine_token(p.y, 0, p.slot_of, p.topk_w, t, p.k, p.H, p.out, 0, lane);
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  gemm_fini<1>(sm);
+}
+
+template <bool kBS, int kBFmt, bool kE4>
+cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
+  const int S = a.T * a.k;
+  const int afmt = a.act == MOE_BF16 ? 0 : 1;
+  const int bfmt = a.wt == MOE_BF16 ? 0 : (a.wt == MOE_E4M3 ? 1 : 2);
+  CUtensorMap tmX, tmW1, tmH, tmW2;
+  if (!make_kmajor_map(&tmX, a.x_perm, S, a.H, afmt) ||
+      !make_kmajor_map(&tmW1, a.w1, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, bfmt) ||
+      !make_kmajor_map(&tmH, a.h, S, a.I, afmt) ||
+      !make_kmajor_map(&tmW2, a.w2, static_cast<uint64_t>(a.E) * a.H, a.I, bfmt))
+    return cudaErrorInvalidValue;
+  FwdParams p;
+  p.x = a.x;
+  p.x_scales = a.x_scales;
+  p.logits = a.logits;
+  p.bias = a.bias;
+  p.sigmoid = a.sigmoid;
+  p.renorm = a.renorm;
+  p.T = a.T;
+  p.H = a.H;
+  p.E = a.E;
+  p.k = a.k;
+  p.C = (a.T + kChunkTokens - 1) / kChunkTokens;
+  p.row_bytes = a.H * (a.act == MOE_BF16 ? 2 : 1);
+  p.topk_idx = a.topk_idx;
+  p.topk_w = a.topk_w;
+  p.offsets = a.offsets;
+  p.perm_src = a.perm_src;
+  p.slot_of = a.slot_of;
+  p.x_perm = a.x_perm;
+  p.x_perm_scales = a.x_perm_scales;
+  p.cnt = a.cnt;
+  p.totals = a.totals;
+  p.y = a.y;
+  p.out = a.out;
+  p.bar = a.bar;
+  p.err = a.err;
+  TcParams l1{}, l2{};
+  l1.offsets = l2.offsets = a.offsets;
+  l1.E = l2.E = a.E;
+  l1.S = l2.S = S;
+  l1.I = l2.I = a.I;
+  l1.err = l2.err = a.err;
+  l1.K = a.H;
+  l1.n_tiles = a.I / 128;
+  l1.w_rows = 2 * a.I;
+  l1.n_out = a.I;
+  l1.a_scales = a.x_perm_scales;
+  l1.b_scales = a.w1_scales;
+  l1.out = a.h;
+  l1.out_scales = a.h_scales;
+  l2.K = a.I;
+  l2.n_tiles = (a.H + kBN - 1) / kBN;
+  l2.w_rows = a.H;
+  l2.n_out = a.H;
+  l2.a_scales = a.h_scales;
+  l2.b_scales = a.w2_scales;
+  l2.out = a.y;
+  l2.out_scales = nullptr;
+  p.l1 = l1;
+  p.l2 = l2;
+
+  auto kern = moe_forward_kernel<kBS, kBFmt, kE4>;
+  const size_t smem = Cfg<1>::kSmem;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), s);
+  if (err != cudaSuccess) return err;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms());
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  count_launch();
+  return cudaLaunchKernelEx(&cfg, kern, tmX, tmW1, tmH, tmW2, p);
+}
+
+}  // namespace
+
+cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s) {
+  // the dispatch phases keep per-warp masks (8 x E words) in the 64 KB of A stages
+  if (a.E > 1024) return cudaErrorNotSupported;
+  if (a.act == MOE_BF16 && a.wt == MOE_BF16) return launch<false, 0, false>(a, s);
+  if (a.act == MOE_E4M3 && a.wt == MOE_E4M3) return launch<true, 0, true>(a, s);
+  if (a.act == MOE_E4M3 && a.wt == MOE_E2M1) return launch<true, 5, true>(a, s);
+  return cudaErrorNotSupported;
+}
+
+}  // namespace moe

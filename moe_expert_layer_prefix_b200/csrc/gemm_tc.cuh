@@ -1,0 +1,689 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// linear-1 (+ SwiGLU + requantisation) and linear-2 of every expert, as the source pages'
+// pipeline lists them (jiqizhixin, "DeepSeek悄悄更新：Mega MoE、FP4 Indexer来了", section
+// "Mega MoE 是什么？", pipeline paragraph; FP8 x FP4 paragraph: FP8 activations with FP4
+// weights; youleyou, "DeepSeek 模型更新解读 Tile Kernels 与 DeepEP V2 新特性", Tile Kernels
+// feature list, quantisation item: FP8 quantisation fused with SwiGLU).
+//
+// Both GEMMs have the form  D[m, n] = sum_k A[m, k] * B[n, k]  per expert, A = the expert's
+// rows of x_perm (or h), B = the expert's K-major weight matrix.  Persistent CTAs (one per
+// SM) walk a static list of output tiles (expert, m-block, n-block) of N = 256 columns.
+// Two tile shapes:
+//   single  one CTA, M = 128: A 128 x 128 B and B 256 x 128 B per k-step, 4 stages
+//   pair    a 2-CTA cluster, M = 256 (tcgen05 cta_group::2): each CTA loads its own 128 A
+//           rows and half of the B rows (128 x 128 B) per k-step, 6 stages; the leader CTA
+//           issues the MMAs, which read both CTAs' shared memory and write both CTAs' TMEM,
+//           so each weight tile crosses L2 -> SM once per 256 rows and each SM moves 32 KB
+//           per k-step instead of 48 KB.
+// Roles per CTA:
+//   warp 0      TMA producer into the shared-memory ring (128-byte swizzle); in a pair, both
+//               CTAs' copies complete on the leader's stage barrier
+//   warp 1      MMA issuer (one thread, leader CTA): tcgen05.mma 128|256 x 256 x {16|32}
+//               into a TMEM fp32 accumulator (256 columns); tcgen05.commit frees ring stages
+//               (in both CTAs of a pair)
+//   warp 2      scale loader (block-scaled kinds): prefetches the raw scale words of each
+//               k-step into a small shared-memory ring
+//   warp 3      scale converter: UE8M0 words in the layout tcgen05.cp reads, then signals the
+//               (leader's) stage barrier; before the first phase it also builds the tile list
+//   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp i reads TMEM lanes 32i..32i+31,
+//               one output row per thread), SwiGLU + BF16 / E4M3 requantisation (linear-1)
+//               or BF16 conversion (linear-2), 16-byte global stores
+//
+// linear-1 tiles take B rows [n*128, n*128+128) (gate) and [I + n*128, ...) (up), so the
+// accumulator holds gate in columns 0..127 and up in 128..255 and each tile yields 128 h
+// columns -- exactly one 1x128 requantisation block per row.
+//
+// Kinds: BF16 x BF16 -> tcgen05.mma kind::f16.  E4M3 x {E4M3, E2M1} -> kind::mxf8f6f4
+// block-scaled with one UE8M0 scale per 32 elements of K: the fp32 power-of-two activation
+// and E4M3 weight scales convert to UE8M0 losslessly; E2M1 weights carry UE8M0 natively.
+// E2M1 tiles are expanded by TMA to one byte per element in shared memory (16U4_ALIGN16B),
+// the operand layout kind::mxf8f6f4 reads, while HBM traffic stays at 4 bits per weight.
+//
+// Shared by the grouped-GEMM kernel and the persistent forward kernel.  Every wait is
+// bounded: a stuck pipeline records MOE_ERR_TIMEOUT with its site in the
+// device error word, raises a CTA-wide abort flag, drains what it issued, frees TMEM and
+// returns.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+namespace gemm {
+
+constexpr int kBM = 128;           // accumulator rows per CTA (TMEM lanes)
+constexpr int kBN = 256;           // accumulator columns (MMA N)
+constexpr int kRowBytes = 128;     // K bytes per tile row per stage (one swizzle atom)
+constexpr int kATileBytes = kBM * kRowBytes;  // 16 KB
+constexpr int kSfaBytes = 512;     // 128 rows x 4 UE8M0
+constexpr int kSfbBytes = 1024;    // 256 rows x 4 UE8M0
+constexpr int kTmemCols = 512;
+constexpr int kAccCol = 0;
+constexpr int kSfaCol = 256;       // scale-factor column sets start here ...
+constexpr int kSfbCol = 260;       // ... SFA (4 columns) then SFB (8 columns)
+constexpr int kSfSetCols = 12;
+constexpr int kSfSets = 4;         // rotated per k-step so a copy never waits on the MMA
+                                   // still reading the previous k-step's scales
+constexpr int kThreads = 256;
+constexpr int kMaxE = 1024;
+constexpr int kMaxStages = 6;
+constexpr int kRawWords = 12;       // raw scale words per lane per k-step (4 A + up to 8 B)
+constexpr int kRawBytes = 32 * kRawWords * 4;
+
+struct TcParams {
+  const int32_t* offsets;  // [E+1]
+  int E, S, K;             // K = reduction length in elements
+  int n_tiles;             // n-blocks per m-block
+  int w_rows;              // weight rows per expert (2I or H)
+  int I;                   // linear-1: offset of the up rows; unused for linear-2
+  int n_out;               // output columns (I for linear-1, H for linear-2)
+  const float* a_scales;   // fp32 [S, K/128] (block-scaled kinds)
+  const void* b_scales;    // E4M3: fp32 [E, w_rows/128, K/128]; E2M1: u8 [E, w_rows, K/32]
+  void* out;
+  float* out_scales;       // linear-1 with E4M3 h
+  int* err;
+};
+
+struct SharedState {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t raw_full[kMaxStages];   // scale words staged by the loader warp
+  uint64_t raw_empty[kMaxStages];  // ... and consumed by the converter warp
+  uint64_t acc_full;
+  uint64_t acc_empty;
+  uint64_t drain;
+  uint32_t tmem_base;
+  int abort;
+  int total_tiles;
+  int mb_start[kMaxE + 1];  // exclusive prefix of m-blocks per expert
+  int offs[kMaxE + 1];
+};
+
+template <int kCta>
+struct Cfg {
+  static constexpr int kStages = kCta == 2 ? 6 : 4;
+  static constexpr int kBRows = kBN / kCta;               // B rows this CTA loads per k-step
+  static constexpr int kBTileBytes = kBRows * kRowBytes;  // 32 KB single, 16 KB pair
+  static constexpr int kTileM = kBM * kCta;               // rows of one tile
+  static constexpr size_t kSmem = 1024 + kStages * (kATileBytes + kBTileBytes) +
+                                  kStages * (kSfaBytes + kSfbBytes) + kStages * kRawBytes +
+                                  sizeof(SharedState);
+};
+
+struct Tile {
+  int e, m0, m_end, nb;
+};
+
+__device__ __forceinline__ Tile decode_tile(const SharedState& ss, int E, int n_tiles, int tile_m,
+                                            int t) {
+  const int mb = t / n_tiles;
+  Tile tile;
+  tile.nb = t - mb * n_tiles;
+  int lo = 0, hi = E;  // mb_start[lo] <= mb < mb_start[hi]
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (ss.mb_start[mid] <= mb) lo = mid; else hi = mid;
+  }
+  tile.e = lo;
+  tile.m0 = ss.offs[lo] + (mb - ss.mb_start[lo]) * tile_m;
+  tile.m_end = ss.offs[lo + 1];
+  return tile;
+}
+
+// silu(g) * u = g * u / (1 + e^-g) with the fast exponential and division (a few ulp; far
+// below the BF16 / E4M3 storage step of h).  For g -> -inf the quotient goes to 0.
+__device__ __forceinline__ float silu_mul(float g, float u) {
+  return __fdividef(g * u, 1.0f + __expf(-g));
+}
+
+// Per-thread pipeline counters.  Each role advances only its own; they carry over from one
+// GEMM phase to the next inside a kernel so that the mbarrier phase parities stay in step.
+struct Pipe {
+  uint32_t prod_it = 0;  // producer: k-steps issued into the ring
+  uint32_t mma_it = 0;   // MMA issuer: k-steps consumed
+  uint32_t tiles = 0;    // MMA issuer / epilogue: accumulator uses
+  uint32_t sf_it = 0;    // scale loader / converter: k-steps staged
+};
+
+// Shared-memory carve-up (1024-byte aligned; identical offsets in both CTAs of a pair).
+struct Smem {
+  uint8_t* sA;
+  uint8_t* sB;
+  uint8_t* sSF;
+  uint8_t* sRaw;
+  SharedState* ss;
+};
+
+template <int kCta>
+__device__ __forceinline__ Smem carve(uint8_t* smem_raw) {
+  using C = Cfg<kCta>;
+  Smem m;
+  m.sA = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                    ~static_cast<uintptr_t>(1023));
+  m.sB = m.sA + C::kStages * kATileBytes;
+  m.sSF = m.sB + C::kStages * C::kBTileBytes;             // per stage: SFA 512 B, SFB 1024 B
+  m.sRaw = m.sSF + C::kStages * (kSfaBytes + kSfbBytes);  // per stage: [lane][kRawWords]
+  m.ss = reinterpret_cast<SharedState*>(m.sRaw + C::kStages * kRawBytes);
+  return m;
+}
+
+// Barriers and TMEM; warps 0 and 1.  The caller synchronises the CTA (and the cluster)
+// before any role starts.
+template <int kCta, bool kBlockScaled>
+__device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tmaps, int ntmaps) {
+  SharedState& ss = *sm.ss;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < Cfg<kCta>::kStages; ++s) {
+      mbar_init(&ss.full[s], 1 + (kBlockScaled ? kCta : 0));
+      mbar_init(&ss.empty[s], 1);
+      mbar_init(&ss.raw_full[s], 1);
+      mbar_init(&ss.raw_empty[s], 1);
+    }
+    mbar_init(&ss.acc_full, 1);
+    mbar_init(&ss.acc_empty, 4 * kCta);
+    mbar_init(&ss.drain, 1);
+    ss.abort = 0;
+    fence_barrier_init();
+    for (int i = 0; i < ntmaps; ++i) tma_prefetch_desc(tmaps + i);
+  }
+  if (warp == 1) {
+    if constexpr (kCta == 2) {
+      tmem_alloc_pair(&ss.tmem_base, kTmemCols);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&ss.tmem_base, kTmemCols);
+      tmem_relinquish();
+    }
+  }
+}
+
+// Tile list of one GEMM from the expert offsets (warp 3; the caller synchronises after).
+template <int kCta>
+__device__ __forceinline__ void gemm_prefix(const Smem& sm, const int32_t* offsets, int E,
+                                            int n_tiles) {
+  using C = Cfg<kCta>;
+  SharedState& ss = *sm.ss;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp != 3) return;
+  int carry = 0;
+  for (int base = 0; base <= E; base += 32) {
+    const int e = base + lane;
+    int o = 0, cnt = 0;
+    if (e <= E) {
+      o = __ldcg(offsets + e);
+      ss.offs[e] = o;
+    }
+    if (e < E) cnt = (__ldcg(offsets + e + 1) - o + C::kTileM - 1) / C::kTileM;
+    int incl = cnt;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    if (e <= E) ss.mb_start[e] = carry + incl - cnt;
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  if (lane == 0) ss.total_tiles = ss.mb_start[E] * n_tiles;
+}
+
+// Releases TMEM (warp 1); the caller synchronises the CTA (and the cluster) first.
+template <int kCta>
+__device__ __forceinline__ void gemm_fini(const Smem& sm) {
+  if ((threadIdx.x >> 5) == 1) {
+    __syncwarp();
+    if constexpr (kCta == 2) tmem_dealloc_pair(sm.ss->tmem_base, kTmemCols);
+    else tmem_dealloc(sm.ss->tmem_base, kTmemCols);
+  }
+}
+
+// One grouped GEMM over the tile list in shared memory (gemm_prefix), all roles.
+// kCta: 1 (single) or 2 (pair).  kBlockScaled: false -> BF16 kind::f16; true ->
+// kind::mxf8f6f4 with A = E4M3 and B = E4M3 (kBFmt 0) or E2M1 (kBFmt 5).  kSwiGLU: linear-1
+// epilogue, else linear-2.  kOutE4M3: linear-1 stores h as E4M3 + 1x128 scales (else BF16).
+template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3>
+__device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
+                                           const TcParams& p, const Smem& sm, Pipe& pipe) {
+  using C = Cfg<kCta>;
+  constexpr bool kPair = kCta == 2;
+  constexpr int kStages = C::kStages;
+  const CUtensorMap& tmA = *tmA_;
+  const CUtensorMap& tmB = *tmB_;
+  uint8_t* sA = sm.sA;
+  uint8_t* sB = sm.sB;
+  uint8_t* sSF = sm.sSF;
+  uint8_t* sRaw = sm.sRaw;
+  SharedState& ss = *sm.ss;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const int cid = kPair ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int ncl = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  constexpr int kElemsPerRow = kBlockScaled ? 128 : 64;  // K elements per stage
+  const int KB = p.K / kElemsPerRow;
+  const uint32_t tmem = ss.tmem_base;
+  const int total = ss.total_tiles;
+  volatile int* abort = &ss.abort;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      constexpr uint32_t kBBytes = kBFmt == 5 ? C::kBTileBytes / 2 : C::kBTileBytes;
+      constexpr uint32_t kCtaBytes = kATileBytes + kBBytes;
+      uint32_t it = pipe.prod_it;
+      const uint32_t it0 = it;
+      for (int t = cid; t < total && !*abort; t += ncl) {
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
+        const int arow = tile.m0 + static_cast<int>(rank) * kBM;
+        // B rows of this CTA: linear-1 gate rows [nb*128, +128) then up rows [I + nb*128, +128);
+        // linear-2 rows [nb*256, +256); a pair splits them between its two CTAs
+        const int ebase = tile.e * p.w_rows;
+        const int g0 = kSwiGLU ? ebase + tile.nb * 128 : ebase + tile.nb * kBN;
+        const int g1 = kSwiGLU ? ebase + p.I + tile.nb * 128 : g0 + 128;
+        const int brow = rank == 0 ? g0 : g1;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int stage = static_cast<int>(it % kStages);
+          const uint32_t phase = (it / kStages) & 1u;
+          if (!mbar_wait<kPair>(&ss.empty[stage], phase ^ 1u, p.err, SITE_GEMM_EMPTY, abort)) break;
+          const int kx = kb * kElemsPerRow;
+          if constexpr (kPair) {
+            if (rank == 0) mbar_arrive_expect_tx(&ss.full[stage], 2 * kCtaBytes);
+            const uint32_t bar = mapa_shared(smem_u32(&ss.full[stage]), 0);
+            tma_load_2d_pair(sA + stage * kATileBytes, &tmA, bar, kx, arow);
+            tma_load_2d_pair(sB + stage * C::kBTileBytes, &tmB, bar, kx, brow);
+          } else {
+            mbar_arrive_expect_tx(&ss.full[stage], kCtaBytes);
+            tma_load_2d(sA + stage * kATileBytes, &tmA, &ss.full[stage], kx, arow);
+            tma_load_2d(sB + stage * C::kBTileBytes, &tmB, &ss.full[stage], kx, g0);
+            tma_load_2d(sB + stage * C::kBTileBytes + C::kBTileBytes / 2, &tmB, &ss.full[stage], kx,
+                        g1);
+          }
+          ++it;
+        }
+      }
+      pipe.prod_it = it;
+      if (*abort && rank == 0) {
+        // drain: wait (bounded) for the copies of the last stages issued into this ring
+        const uint32_t issued = it - it0;
+        const uint32_t n = issued < static_cast<uint32_t>(kStages) ? issued : kStages;
+        for (uint32_t i = 1; i <= n; ++i) {
+          const int stage = static_cast<int>((it - i) % kStages);
+          const uint32_t phase = ((it - i) / kStages) & 1u;
+          const long long t0 = clock64();
+          while (!mbar_try_wait_scoped<kPair>(&ss.full[stage], phase)) {
+            if (clock64() - t0 > kWaitLimitCycles) {
+              report_error(p.err, MOE_ERR_TIMEOUT, SITE_GEMM_DRAIN);
+              break;
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0 && rank == 0) {
+      constexpr int kMmaM = kBM * kCta;
+      constexpr uint32_t kIdesc = kBlockScaled ? idesc_mxf8f6f4(kMmaM, kBN, 0u, kBFmt)
+                                               : idesc_bf16(kMmaM, kBN);
+      uint32_t it = pipe.mma_it, tiles = pipe.tiles;
+      bool issued_any = false;
+      for (int t = cid; t < total && !*abort; t += ncl) {
+        const uint32_t acc_phase = tiles & 1u;
+        if (!mbar_wait<kPair>(&ss.acc_empty, acc_phase ^ 1u, p.err, SITE_GEMM_ACC_EMPTY, abort))
+          break;
+        tc_fence_after();
+        bool ok = true;
+        for (int kb = 0; kb < KB; ++kb) {
+          const int stage = static_cast<int>(it % kStages);
+          const uint32_t phase = (it / kStages) & 1u;
+          if (!mbar_wait<kPair>(&ss.full[stage], phase, p.err, SITE_GEMM_FULL, abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * kATileBytes));
+          const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
+          const uint32_t sfset = it % kSfSets;
+          const uint32_t tsfa = tmem + kSfaCol + sfset * kSfSetCols;
+          const uint32_t tsfb = tmem + kSfbCol + sfset * kSfSetCols;
+          if constexpr (kBlockScaled) {
+            const uint32_t sf = smem_u32(sSF + stage * (kSfaBytes + kSfbBytes));
+            if constexpr (kPair) {
+              tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sf));
+              tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sf + kSfaBytes));
+              tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+            } else {
+              tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sf));
+              tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sf + kSfaBytes));
+              tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+            }
+          }
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks) {
+            // advance 32 bytes of K inside the 128-byte swizzle atom
+            const uint64_t ad = adesc + static_cast<uint64_t>(ks * 2);
+            const uint64_t bd = bdesc + static_cast<uint64_t>(ks * 2);
+            const uint32_t acc = (kb | ks) != 0 ? 1u : 0u;
+            if constexpr (kBlockScaled) {
+              const uint32_t id = kIdesc | (static_cast<uint32_t>(ks) << 4) |
+                                  (static_cast<uint32_t>(ks) << 29);
+              const uint32_t sfa = tsfa | (static_cast<uint32_t>(ks) << 30);
+              const uint32_t sfb = tsfb | (static_cast<uint32_t>(ks) << 30);
+              if constexpr (kPair) mma_mxf8f6f4_pair(tmem + kAccCol, ad, bd, id, sfa, sfb, acc);
+              else mma_mxf8f6f4(tmem + kAccCol, ad, bd, id, sfa, sfb, acc);
+            } else {
+              if constexpr (kPair) mma_bf16_pair(tmem + kAccCol, ad, bd, kIdesc, acc);
+              else mma_bf16(tmem + kAccCol, ad, bd, kIdesc, acc);
+            }
+          }
+          issued_any = true;
+          if constexpr (kPair) tc_commit_pair(&ss.empty[stage], 0x3);
+          else tc_commit(&ss.empty[stage]);
+          ++it;
+        }
+        if (!ok) break;
+        if constexpr (kPair) tc_commit_pair(&ss.acc_full, 0x3);
+        else tc_commit(&ss.acc_full);
+        ++tiles;
+      }
+      pipe.mma_it = it;
+      pipe.tiles = tiles;
+      if (*abort && issued_any) {
+        // let the issued MMAs finish before TMEM is released
+        if constexpr (kPair) tc_commit_pair(&ss.drain, 0x1);
+        else tc_commit(&ss.drain);
+        const long long t0 = clock64();
+        while (!mbar_try_wait_scoped<kPair>(&ss.drain, 0)) {
+          if (clock64() - t0 > kWaitLimitCycles) break;
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------------ scale loader
+    // Iterations i = (tile, k-step) of this CTA in order.  The raw scale words of iteration
+    // i + kSfDepth are loaded right after iteration i is staged, so their latency overlaps
+    // kSfDepth k-steps; row pointers are set up once per tile.  Words are staged in a small
+    // shared-memory ring for the converter warp, which therefore never has global loads in
+    // flight when it signals the (pair leader's) stage barrier.
+    if constexpr (kBlockScaled) {
+      constexpr int kSfDepth = 4;
+      constexpr int kNB = kBFmt == 5 ? 8 : 2;  // B words per lane per k-step
+      const int KS = p.K / 128;                // fp32 scale columns of A (and of E4M3 B)
+      uint32_t ra[kSfDepth][4];
+      uint32_t rb[kSfDepth][kNB];
+      int lt = cid, lkb = 0;  // loader state: the next (tile, k-step) to load
+      const float* pa[4];
+      const uint8_t* pb[kNB];
+      auto setup_tile = [&]() {
+        if (lt >= total) return;
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) {
+          int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * r1;
+          m = m < p.S ? m : p.S - 1;  // rows past S are zero-filled by TMA; any scale will do
+          pa[r1] = p.a_scales + static_cast<size_t>(m) * KS;
+        }
+        const int wr0 = kSwiGLU ? tile.nb * 128 : tile.nb * kBN;     // first B row, atom 0
+        const int wr1 = kSwiGLU ? p.I + tile.nb * 128 : wr0 + 128;   // first B row, atom 1
+        if constexpr (kBFmt == 5) {
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int r1 = 0; r1 < 4; ++r1) {
+              int wr = (a == 0 ? wr0 : wr1) + lane + 32 * r1;
+              wr = wr < p.w_rows ? wr : p.w_rows - 1;
+              pb[a * 4 + r1] = static_cast<const uint8_t*>(p.b_scales) +
+                               (static_cast<size_t>(tile.e) * p.w_rows + wr) * (p.K / 32);
+            }
+        } else {
+#pragma unroll
+          for (int a = 0; a < 2; ++a) {
+            int wr = a == 0 ? wr0 : wr1;
+            wr = wr < p.w_rows ? wr : p.w_rows - 1;
+            pb[a] = reinterpret_cast<const uint8_t*>(
+                static_cast<const float*>(p.b_scales) +
+                (static_cast<size_t>(tile.e) * (p.w_rows / 128) + wr / 128) * KS);
+          }
+        }
+      };
+      auto load_next = [&](uint32_t (&a4)[4], uint32_t (&bw)[kNB]) {
+        if (lt >= total) return;
+#pragma unroll
+        for (int r1 = 0; r1 < 4; ++r1) a4[r1] = __float_as_uint(__ldcg(pa[r1] + lkb));
+        if constexpr (kBFmt == 5) {
+#pragma unroll
+          for (int r = 0; r < 8; ++r) bw[r] = __ldg(reinterpret_cast<const uint32_t*>(pb[r] + lkb * 4));
+        } else {
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+            bw[a] = __float_as_uint(__ldg(reinterpret_cast<const float*>(pb[a]) + lkb));
+        }
+        if (++lkb == KB) {
+          lkb = 0;
+          lt += ncl;
+          setup_tile();
+        }
+      };
+      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
+      const int n_iter = my_tiles * KB;
+      setup_tile();
+#pragma unroll
+      for (int j = 0; j < kSfDepth; ++j) load_next(ra[j], rb[j]);
+      bool ok = true;
+      const uint32_t it0 = pipe.sf_it;
+      for (int base = 0; base < n_iter && ok; base += kSfDepth) {
+#pragma unroll
+        for (int j = 0; j < kSfDepth; ++j) {
+          const int i = base + j;
+          if (i >= n_iter) break;
+          const int stage = static_cast<int>((it0 + i) % kStages);
+          const uint32_t phase = ((it0 + i) / kStages) & 1u;
+          if (!mbar_wait(&ss.raw_empty[stage], phase ^ 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) {
+            ok = false;
+            break;
+          }
+          uint32_t* raw = reinterpret_cast<uint32_t*>(sRaw + stage * kRawBytes) + lane * kRawWords;
+          *reinterpret_cast<uint4*>(raw) = make_uint4(ra[j][0], ra[j][1], ra[j][2], ra[j][3]);
+          if constexpr (kBFmt == 5) {
+            *reinterpret_cast<uint4*>(raw + 4) = make_uint4(rb[j][0], rb[j][1], rb[j][2], rb[j][3]);
+            *reinterpret_cast<uint4*>(raw + 8) = make_uint4(rb[j][4], rb[j][5], rb[j][6], rb[j][7]);
+          } else {
+            *reinterpret_cast<uint2*>(raw + 4) = make_uint2(rb[j][0], rb[j][1]);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ss.raw_full[stage]);
+          load_next(ra[j], rb[j]);
+        }
+      }
+      pipe.sf_it = it0 + n_iter;
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------------ scale converter
+    // Turns the staged fp32 / UE8M0 words into the shared-memory layout tcgen05.cp reads
+    // (32 rows x 16 bytes per 128-row atom: byte 16*(r%32) + 4*(r/32) + k-sub-block) and
+    // signals the stage barrier of the pair leader.
+    if constexpr (kBlockScaled) {
+      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
+      const int n_iter = my_tiles * KB;
+      const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.full[0]), 0);
+      const uint32_t it0 = pipe.sf_it;
+      for (int i = 0; i < n_iter; ++i) {
+        const int stage = static_cast<int>((it0 + i) % kStages);
+        const uint32_t phase = ((it0 + i) / kStages) & 1u;
+        if (!mbar_wait(&ss.raw_full[stage], phase, p.err, SITE_GEMM_SF_EMPTY, abort)) break;
+        if (!mbar_wait<kPair>(&ss.empty[stage], phase ^ 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) break;
+        const uint32_t* raw = reinterpret_cast<const uint32_t*>(sRaw + stage * kRawBytes) + lane * kRawWords;
+        const uint4 ra4 = *reinterpret_cast<const uint4*>(raw);
+        uint32_t b8[8];
+        if constexpr (kBFmt == 5) {
+          const uint4 lo = *reinterpret_cast<const uint4*>(raw + 4);
+          const uint4 hi = *reinterpret_cast<const uint4*>(raw + 8);
+          b8[0] = lo.x; b8[1] = lo.y; b8[2] = lo.z; b8[3] = lo.w;
+          b8[4] = hi.x; b8[5] = hi.y; b8[6] = hi.z; b8[7] = hi.w;
+        } else {
+          const uint2 w2 = *reinterpret_cast<const uint2*>(raw + 4);
+          const uint32_t v0 = ((w2.x >> 23) & 0xFFu) * 0x01010101u;
+          const uint32_t v1 = ((w2.y >> 23) & 0xFFu) * 0x01010101u;
+          b8[0] = b8[1] = b8[2] = b8[3] = v0;
+          b8[4] = b8[5] = b8[6] = b8[7] = v1;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ss.raw_empty[stage]);
+        // fp32 power-of-two scale -> its UE8M0 byte (the biased exponent), x4 along K
+        const uint32_t a0 = ((ra4.x >> 23) & 0xFFu) * 0x01010101u;
+        const uint32_t a1 = ((ra4.y >> 23) & 0xFFu) * 0x01010101u;
+        const uint32_t a2 = ((ra4.z >> 23) & 0xFFu) * 0x01010101u;
+        const uint32_t a3 = ((ra4.w >> 23) & 0xFFu) * 0x01010101u;
+        uint8_t* sf = sSF + stage * (kSfaBytes + kSfbBytes);
+        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(a0, a1, a2, a3);
+        *reinterpret_cast<uint4*>(sf + kSfaBytes + 16 * lane) = make_uint4(b8[0], b8[1], b8[2], b8[3]);
+        *reinterpret_cast<uint4*>(sf + kSfaBytes + 512 + 16 * lane) =
+            make_uint4(b8[4], b8[5], b8[6], b8[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(full_lead0 + stage * sizeof(uint64_t));
+          else mbar_arrive(&ss.full[stage]);
+        }
+      }
+      pipe.sf_it = it0 + n_iter;
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp - 4;  // TMEM lane quadrant
+    const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
+    uint32_t tiles = pipe.tiles;
+    const uint32_t acc_empty_lead = mapa_shared(smem_u32(&ss.acc_empty), 0);
+    for (int t = cid; t < total && !*abort; t += ncl) {
+      const uint32_t acc_phase = tiles & 1u;
+      const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
+      // every lane waits; the decision is made warp-uniform so that the .sync.aligned
+      // TMEM loads below always run with the full warp
+      const bool ready =
+          mbar_wait<kPair>(&ss.acc_full, acc_phase, p.err, SITE_GEMM_ACC_FULL, abort);
+      if (!__all_sync(0xffffffffu, ready)) break;
+      tc_fence_after();
+      const int row = tile.m0 + static_cast<int>(rank) * kBM + q * 32 + lane;
+      const bool valid = row < tile.m_end;
+      if constexpr (kSwiGLU) {
+        if constexpr (kOutE4M3) {
+          float h[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(trow + kAccCol + 32 * c, g);
+            tmem_ld32(trow + kAccCol + 128 + 32 * c, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              h[32 * c + i] = silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]));
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
+          else mbar_arrive(&ss.acc_empty);
+        }
+          float amax = 0.0f;
+#pragma unroll
+          for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(h[i]));
+          const int e = max(e4m3_scale_exponent(amax), -126);
+          const float inv = exp2i(-e);
+          if (valid) {
+            uint8_t* dst = static_cast<uint8_t*>(p.out) + static_cast<size_t>(row) * p.n_out +
+                           tile.nb * 128;
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int b = 16 * v + 4 * i;
+                const __nv_fp8x2_storage_t lo =
+                    __nv_cvt_float2_to_fp8x2(make_float2(h[b] * inv, h[b + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t hi =
+                    __nv_cvt_float2_to_fp8x2(make_float2(h[b + 2] * inv, h[b + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+                w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+              }
+              reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            p.out_scales[static_cast<size_t>(row) * (p.n_out / 128) + tile.nb] = exp2i(e);
+          }
+        } else {
+          uint32_t w[64];  // 128 h values as BF16 pairs
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(trow + kAccCol + 32 * c, g);
+            tmem_ld32(trow + kAccCol + 128 + 32 * c, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                  silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
+                  silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
+              w[16 * c + i] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
+          else mbar_arrive(&ss.acc_empty);
+        }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                  static_cast<size_t>(row) * p.n_out + tile.nb * 128);
+#pragma unroll
+            for (int v = 0; v < 16; ++v)
+              dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
+        }
+      } else {
+        // pack the whole row to BF16 in registers, hand TMEM back, then store
+        uint32_t w[kBN / 2];
+#pragma unroll
+        for (int c = 0; c < kBN / 32; c += 2) {  // two 32-column loads per wait
+          uint32_t d0[32], d1[32];
+          tmem_ld32(trow + kAccCol + 32 * c, d0);
+          tmem_ld32(trow + kAccCol + 32 * (c + 1), d1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 b0 =
+                __floats2bfloat162_rn(__uint_as_float(d0[2 * i]), __uint_as_float(d0[2 * i + 1]));
+            const __nv_bfloat162 b1 =
+                __floats2bfloat162_rn(__uint_as_float(d1[2 * i]), __uint_as_float(d1[2 * i + 1]));
+            w[16 * c + i] = *reinterpret_cast<const uint32_t*>(&b0);
+            w[16 * (c + 1) + i] = *reinterpret_cast<const uint32_t*>(&b1);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
+          else mbar_arrive(&ss.acc_empty);
+        }
+        if (valid) {
+          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(row) * p.n_out;
+#pragma unroll
+          for (int c = 0; c < kBN / 32; ++c) {
+            const int col = tile.nb * kBN + 32 * c;
+            if (col < p.n_out) {
+              uint4* dst = reinterpret_cast<uint4*>(orow + col);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                dst[v] = make_uint4(w[16 * c + 4 * v], w[16 * c + 4 * v + 1], w[16 * c + 4 * v + 2],
+                                    w[16 * c + 4 * v + 3]);
+            }
+          }
+        }
+      }
+      ++tiles;
+    }
+    pipe.tiles = tiles;
+  }
+
+}
+
+}  // namespace gemm
+}  // namespace moe

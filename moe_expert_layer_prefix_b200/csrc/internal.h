@@ -50,6 +50,41 @@ cudaError_t launch_linear2_simt(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s);
 
+// 2-D K-major tensor map: rows x K, box {128-byte K slice, 128 rows}, 128-byte swizzle.
+// fmt: 0 = BF16, 1 = 8-bit, 2 = E2M1 (expanded to one byte per element in shared memory).
+bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int fmt);
+
+// The whole layer in one persistent cooperative launch (tensor-core formats only);
+// returns cudaErrorNotSupported when the layer cannot run that way.
+struct ForwardArgs {
+  const void* x;
+  const float* x_scales;
+  const float* logits;
+  const float* bias;
+  int sigmoid, renorm, T, H, E, k, I;
+  int act, wt;
+  const void* w1;
+  const void* w1_scales;
+  const void* w2;
+  const void* w2_scales;
+  int32_t* topk_idx;
+  float* topk_w;
+  int32_t* offsets;
+  int32_t* perm_src;
+  int32_t* slot_of;
+  void* x_perm;
+  float* x_perm_scales;
+  int32_t* cnt;      // dispatch chunk counts [C][E]
+  int32_t* totals;   // [E]
+  void* h;
+  float* h_scales;
+  void* y;
+  void* out;
+  uint32_t* bar;     // grid barrier words (zeroed by the launcher)
+  int* err;
+};
+cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s);
+
 int* device_error_word();   // device address of the calling device's error word
 int gemm_tile_mode();       // 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles
 int num_sms();

@@ -1,0 +1,155 @@
+// Router, per token: one warp selects the k best experts and writes their gates (shared by
+// the router kernel and the persistent forward kernel).
+//
+// Gating as the source pages list it (youleyou, "DeepSeek 模型更新解读 Tile Kernels 与 DeepEP
+// V2 新特性", section "Tile Kernels：逼近硬件极限的底层优化": gating = top-k expert
+// selection with scoring; routing = weight normalisation).  The scoring rules are the
+// library's reading of that item:
+//   softmax: key = logit; gate_j = exp(l_j - l_0) / sum over the selected (renorm) or over
+//            all experts (no renorm), l_0 the largest logit;
+//   sigmoid: s = 1 / (1 + exp(-l)) evaluated as a fixed sequence of correctly rounded fp32
+//            operations (the exponential below), key = s + bias_e;
+//            gate_j = s_j / sum of selected s (renorm) or s_j.
+// Rank order: key descending, equal keys -> lower expert id.
+//
+// HBM-bound: each token's E logits are read once, coalesced across the warp.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+// fp32 exponential by Cody-Waite range reduction (two-part ln 2) and the degree-7 Taylor
+// polynomial of the reduced argument, every step a separately rounded fp32 operation
+// (Cody & Waite, "Software Manual for the Elementary Functions", 1980).  Used only to form
+// the sigmoid router's selection keys, so that the selection is a function of the fp32
+// keys alone.
+__device__ __forceinline__ float exp_keys_f32(float x) {
+  const float kLog2e = 1.44269504088896340736f;
+  const float kLn2Hi = 0.693145751953125f;
+  const float kLn2Lo = 1.42860682030941723212e-6f;
+  x = fminf(fmaxf(x, -80.0f), 80.0f);
+  const float n = rintf(__fmul_rn(x, kLog2e));
+  float r = __fsub_rn(x, __fmul_rn(n, kLn2Hi));
+  r = __fsub_rn(r, __fmul_rn(n, kLn2Lo));
+  float p = 1.98412698412698412698e-4f;                 // 1/7!
+  p = __fadd_rn(__fmul_rn(p, r), 1.38888888888888888889e-3f);  // 1/6!
+  p = __fadd_rn(__fmul_rn(p, r), 8.33333333333333333333e-3f);  // 1/5!
+  p = __fadd_rn(__fmul_rn(p, r), 4.16666666666666666667e-2f);  // 1/4!
+  p = __fadd_rn(__fmul_rn(p, r), 1.66666666666666666667e-1f);  // 1/3!
+  p = __fadd_rn(__fmul_rn(p, r), 0.5f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  p = __fadd_rn(__fmul_rn(p, r), 1.0f);
+  return __fmul_rn(p, exp2i(static_cast<int>(n)));
+}
+
+__device__ __forceinline__ float sigmoid_keys_f32(float l) {
+  return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_keys_f32(-l)));
+}
+
+// (key, id) ordering: larger key first, then lower id.
+__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
+  return ka > kb || (ka == kb && ia < ib);
+}
+
+// One warp selects the k experts of token t and writes topk_idx[t, :], topk_w[t, :].
+// Lanes hold experts lane, lane+32, ...; all 32 lanes must call it together.
+template <int NPL>  // experts per lane (E <= 32 * NPL)
+__device__ __forceinline__ void route_token(const float* __restrict__ logits,
+                                            const float* __restrict__ bias, int t, int E, int k,
+                                            int sigmoid, int renorm,
+                                            int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_w, int lane) {
+  const float* row = logits + static_cast<size_t>(t) * E;
+
+  float key[NPL];
+  float val[NPL];  // softmax: the logit; sigmoid: s
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E) {
+      const float l = __ldg(row + e);
+      if (sigmoid) {
+        const float s = sigmoid_keys_f32(l);
+        val[i] = s;
+        key[i] = __fadd_rn(s, bias ? __ldg(bias + e) : 0.0f);
+      } else {
+        val[i] = l;
+        key[i] = l;
+      }
+    } else {
+      val[i] = 0.0f;
+      key[i] = -INFINITY;
+    }
+  }
+
+  uint32_t taken = 0;
+  int my_idx = 0;      // lane j keeps the j-th selection
+  float my_val = 0.0f;
+  float top_val = 0.0f;
+  for (int j = 0; j < k; ++j) {
+    float bk = -INFINITY;
+    int bi = 0x7FFFFFFF;
+    float bv = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u) && better(key[i], e, bk, bi)) {
+        bk = key[i];
+        bi = e;
+        bv = val[i];
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      if (better(ok, oi, bk, bi)) {
+        bk = ok;
+        bi = oi;
+        bv = ov;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == j) {
+      my_idx = bi;
+      my_val = bv;
+    }
+    if (j == 0) top_val = bv;
+  }
+
+  float g;
+  if (sigmoid) {
+    g = (lane < k) ? my_val : 0.0f;
+    if (renorm) {
+      float sum = g;
+      // rank-order sum: lanes 0..k-1 hold the selected s in rank order
+      float acc = 0.0f;
+      for (int j = 0; j < k; ++j) acc += __shfl_sync(0xffffffffu, sum, j);
+      g = g / acc;
+    }
+  } else {
+    float num = (lane < k) ? expf(my_val - top_val) : 0.0f;
+    float den = 0.0f;
+    if (renorm) {
+      for (int j = 0; j < k; ++j) den += __shfl_sync(0xffffffffu, num, j);
+    } else {
+      float part = 0.0f;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i)
+        if (lane + 32 * i < E) part += expf(val[i] - top_val);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+      den = part;
+    }
+    g = num / den;
+  }
+  if (lane < k) {
+    topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
+    topk_w[static_cast<size_t>(t) * k + lane] = g;
+  }
+}
+
+
+}  // namespace moe

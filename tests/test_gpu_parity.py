@@ -220,17 +220,30 @@ def test_forward_end_to_end(name):
     assert_parity(host_values(out, None, fmt), r["out"], fmt, TOL[wl.act])
 
 
-def test_forward_equals_unfused_chain():
-    wl = SMALL["v3_fp8"]
+@pytest.mark.parametrize("name", ["v3_fp8", "skewed_fp8_fp4", "mixtral_bf16",
+                                  "v3_fp8_pair", "skewed_fp8_fp4_pair"])
+def test_forward_equals_unfused_chain(name):
+    """moe_forward (one persistent launch) produces exactly the bytes of the chain of entry
+    points (same device code, same tile order; single-CTA tiles for both)."""
+    wl = SMALL[name]
     d = _inputs(wl)
     W = weights_of(wl, d)
-    out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
-                        x_scales=d["x_scales"])
-    idx, w = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
-    r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
-    y = M.moe_fused_ffn(r["x_perm"], r["expert_offsets"], W, x_perm_scales=r["x_perm_scales"])
-    out2 = M.moe_combine(y, r["slot_of"], w)
-    assert torch.equal(out, out2)                  # same kernels, same order: bitwise equal
+    M.moe_set_gemm_tiles("single")
+    try:
+        idx1 = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
+        out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
+                            x_scales=d["x_scales"], topk_idx=idx1)
+        idx, w = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+        r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+        y = M.moe_fused_ffn(r["x_perm"], r["expert_offsets"], W,
+                            x_perm_scales=r["x_perm_scales"])
+        out2 = M.moe_combine(y, r["slot_of"], w)
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error()[0] == 0
+    finally:
+        M.moe_set_gemm_tiles("auto")
+    assert torch.equal(idx1, idx)
+    assert torch.equal(out, out2)
 
 
 def test_forward_deterministic():
