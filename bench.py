@@ -353,8 +353,9 @@ def run_native(args, ws, rank, local):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "path": "moe_forward with pinned host in/out"},
         "gpu_launches": int(launches),
-        "gpu_launches_note": "library kernel launches in the headline timed region (the "
-                             "per-stage breakdown loop adds 8 per step)",
+        "gpu_launches_note": "library kernel launches in the headline timed region (one "
+                             "persistent kernel per step; the per-stage breakdown loop "
+                             "runs the chain of entry points, 9 launches per step)",
         "clocks": clk,
     }
     if ws == 1 and not args.no_cpu_baseline:

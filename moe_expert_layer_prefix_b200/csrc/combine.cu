@@ -7,14 +7,39 @@
 namespace moe {
 namespace {
 
-__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y, int y_f32,
+template <bool kF32>
+__global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y,
                                                       const int32_t* __restrict__ slot_of,
                                                       const float* __restrict__ topk_w, int T,
-                                                      int k, int H, void* __restrict__ out,
-                                                      int out_f32) {
+                                                      int k, int H, void* __restrict__ out) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  combine_token(y, y_f32, slot_of, topk_w, t, k, H, out, out_f32, threadIdx.x & 31);
+  combine_token<kF32>(y, slot_of, topk_w, t, k, H, out, threadIdx.x & 31);
+}
+
+// Mixed formats (BF16 y into fp32 out or the reverse) take this simple path.
+__global__ void __launch_bounds__(256) combine_mixed_kernel(const void* __restrict__ y, int y_f32,
+                                                            const int32_t* __restrict__ slot_of,
+                                                            const float* __restrict__ topk_w,
+                                                            int T, int k, int H,
+                                                            void* __restrict__ out, int out_f32) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  for (int c = lane; c < H; c += 32) {
+    float acc = 0.0f;
+    for (int j = 0; j < k; ++j) {
+      const int slot = __ldcg(slot_of + static_cast<size_t>(t) * k + j);
+      const float w = __ldcg(topk_w + static_cast<size_t>(t) * k + j);
+      const size_t i = static_cast<size_t>(slot) * H + c;
+      const float v = y_f32 ? __ldcg(static_cast<const float*>(y) + i)
+                            : __bfloat162float(static_cast<const __nv_bfloat16*>(y)[i]);
+      acc = fmaf(w, v, acc);
+    }
+    const size_t o = static_cast<size_t>(t) * H + c;
+    if (out_f32) static_cast<float*>(out)[o] = acc;
+    else static_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(acc);
+  }
 }
 
 }  // namespace
@@ -23,8 +48,13 @@ cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, con
                            int T, int k, int H, void* out, int out_f32, cudaStream_t s) {
   const int warps = 8;
   count_launch();
-  combine_kernel<<<(T + warps - 1) / warps, 32 * warps, 0, s>>>(y, y_f32, slot_of, topk_w, T, k,
-                                                                H, out, out_f32);
+  const dim3 grid((T + warps - 1) / warps), block(32 * warps);
+  if (y_f32 && out_f32)
+    combine_kernel<true><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out);
+  else if (!y_f32 && !out_f32)
+    combine_kernel<false><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out);
+  else
+    combine_mixed_kernel<<<grid, block, 0, s>>>(y, y_f32, slot_of, topk_w, T, k, H, out, out_f32);
   return cudaGetLastError();
 }
 

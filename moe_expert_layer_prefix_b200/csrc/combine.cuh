@@ -13,68 +13,98 @@
 
 namespace moe {
 
-__device__ __forceinline__ void load8(const void* base, size_t elem, int f32, float (&v)[8]) {
-  if (f32) {
-    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
-    const float4 a = __ldcg(p), b = __ldcg(p + 1);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
-    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
-  } else {
-    const uint4 u = __ldcg(reinterpret_cast<const uint4*>(
-        static_cast<const __nv_bfloat16*>(base) + elem));
-    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 f = __bfloat1622float2(h[i]);
-      v[2 * i] = f.x;
-      v[2 * i + 1] = f.y;
-    }
-  }
-}
-
-// One warp computes out[t, :] (all 32 lanes call it together).
-__device__ __forceinline__ void combine_token(const void* __restrict__ y, int y_f32,
+// One warp computes out[t, :] (all 32 lanes call it together).  y and out are BF16, or fp32
+// for the fp32 layer.  Each lane owns 8 consecutive columns per pass and a warp iteration
+// covers kV passes; the k source rows are read as groups of kJ x kV independent 16-byte
+// loads issued back to back (raw words, converted only afterwards), so a warp keeps many
+// loads in flight even when only a few warps per SM run it.
+template <bool kF32, int kV = 1>
+__device__ __forceinline__ void combine_token(const void* __restrict__ y,
                                               const int32_t* __restrict__ slot_of,
                                               const float* __restrict__ topk_w, int t, int k,
-                                              int H, void* __restrict__ out, int out_f32,
-                                              int lane) {
+                                              int H, void* __restrict__ out, int lane) {
+  constexpr int kJ = 8;
+  constexpr int kWords = kF32 ? 2 : 1;  // 16-byte words per 8 columns
   int my_slot = 0;
   float my_w = 0.0f;
   if (lane < k) {
     my_slot = __ldcg(slot_of + static_cast<size_t>(t) * k + lane);
     my_w = __ldcg(topk_w + static_cast<size_t>(t) * k + lane);
   }
-  const int nvec = H / 8;  // 8 elements per lane per step
-  // The trip count is the same for every lane (shuffles below need the full warp); lanes
-  // past the row's end only skip their loads and stores.
-  for (int v0 = 0; v0 < nvec; v0 += 32) {
-    const int v = v0 + lane;
-    const bool act = v < nvec;
-    float acc[8];
+  const int nvec = H / 8;
+  const uint4* y4 = static_cast<const uint4*>(y);
+  const size_t row_words = static_cast<size_t>(H) / 8 * kWords;
+  // The trip counts are the same for every lane (the shuffles need the full warp); lanes
+  // past the row's end read column 0 and drop the result.
+  for (int v0 = 0; v0 < nvec; v0 += 32 * kV) {
+    size_t col[kV];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
-    for (int j = 0; j < k; ++j) {
-      const int slot = __shfl_sync(0xffffffffu, my_slot, j);
-      const float w = __shfl_sync(0xffffffffu, my_w, j);
-      if (act) {
-        float r[8];
-        load8(y, static_cast<size_t>(slot) * H + static_cast<size_t>(v) * 8, y_f32, r);
+    for (int p = 0; p < kV; ++p) {
+      const int v = v0 + 32 * p + lane;
+      col[p] = static_cast<size_t>(v < nvec ? v : 0) * kWords;
+    }
+    float acc[kV][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, r[i], acc[i]);
+    for (int p = 0; p < kV; ++p)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[p][i] = 0.0f;
+    for (int j0 = 0; j0 < k; j0 += kJ) {
+      uint4 raw[kJ][kV][kWords];
+      float w[kJ];
+      int slot[kJ];
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj) {
+        slot[jj] = __shfl_sync(0xffffffffu, my_slot, (j0 + jj) & 31);
+        w[jj] = __shfl_sync(0xffffffffu, my_w, (j0 + jj) & 31);
+      }
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj) {
+        const uint4* row = y4 + static_cast<size_t>(slot[jj]) * row_words;
+#pragma unroll
+        for (int p = 0; p < kV; ++p)
+#pragma unroll
+          for (int q = 0; q < kWords; ++q) raw[jj][p][q] = __ldcg(row + col[p] + q);
+      }
+#pragma unroll
+      for (int jj = 0; jj < kJ; ++jj) {
+        if (j0 + jj >= k) break;  // warp-uniform
+#pragma unroll
+        for (int p = 0; p < kV; ++p) {
+          float r[8];
+          if constexpr (kF32) {
+            const float* f = reinterpret_cast<const float*>(raw[jj][p]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) r[i] = f[i];
+          } else {
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw[jj][p][0]);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = __bfloat1622float2(h2[i]);
+              r[2 * i] = f.x;
+              r[2 * i + 1] = f.y;
+            }
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) acc[p][i] = fmaf(w[jj], r[i], acc[p][i]);
+        }
       }
     }
-    if (!act) continue;
-    const size_t o = static_cast<size_t>(t) * H + static_cast<size_t>(v) * 8;
-    if (out_f32) {
-      float4* p = reinterpret_cast<float4*>(static_cast<float*>(out) + o);
-      p[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      p[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    } else {
-      uint4 u;
-      __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + o) = u;
+    for (int p = 0; p < kV; ++p) {
+      const int v = v0 + 32 * p + lane;
+      if (v >= nvec) continue;
+      const size_t o = static_cast<size_t>(t) * H + static_cast<size_t>(v) * 8;
+      if constexpr (kF32) {
+        float4* q = reinterpret_cast<float4*>(static_cast<float*>(out) + o);
+        q[0] = make_float4(acc[p][0], acc[p][1], acc[p][2], acc[p][3]);
+        q[1] = make_float4(acc[p][4], acc[p][5], acc[p][6], acc[p][7]);
+      } else {
+        uint4 u;
+        __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[p][2 * i], acc[p][2 * i + 1]);
+        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + o) = u;
+      }
     }
   }
 }

@@ -1,5 +1,5 @@
 // Dispatch kernels (dispatch.cuh holds the per-chunk steps, their ordering rule and their
-// source): hist -> scan -> offsets -> scatter.
+// source): hist -> scan -> offsets -> slots -> row copies.
 #include "common.cuh"
 #include "dispatch.cuh"
 #include "internal.h"
@@ -31,19 +31,26 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
   offsets_from_totals(totals, E, offsets, wsum);
 }
 
-__global__ void __launch_bounds__(32 * kWarps) scatter_kernel(
-    const uint8_t* __restrict__ x, const float* __restrict__ x_scales, int row_bytes, int nscale,
+__global__ void __launch_bounds__(32 * kWarps) slots_kernel(
     const int32_t* __restrict__ topk_idx, int T, int E, int k, int C,
     const int32_t* __restrict__ bases, const int32_t* __restrict__ offsets,
-    uint8_t* __restrict__ x_perm, float* __restrict__ x_perm_scales,
     int32_t* __restrict__ perm_src, int32_t* __restrict__ slot_of) {
   extern __shared__ uint32_t smask[];
-  __shared__ int32_t sslot[kWarps][kChunkTokens][32];
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x * kWarps + w;
   if (chunk >= C) return;
-  scatter_chunk(smask + w * E, sslot[w], x, x_scales, row_bytes, nscale, topk_idx, T, E, k, chunk,
-                bases, offsets, x_perm, x_perm_scales, perm_src, slot_of, lane);
+  assign_slots_chunk(smask + w * E, topk_idx, T, E, k, chunk, bases, offsets, perm_src, slot_of,
+                     lane);
+}
+
+__global__ void __launch_bounds__(256) copy_rows_kernel(
+    const uint8_t* __restrict__ x, const float* __restrict__ x_scales, int row_bytes, int nscale,
+    const int32_t* __restrict__ slot_of, int T, int k, uint8_t* __restrict__ x_perm,
+    float* __restrict__ x_perm_scales) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  copy_token_rows(x, x_scales, row_bytes, nscale, slot_of, t, k, x_perm, x_perm_scales,
+                  threadIdx.x & 31);
 }
 
 }  // namespace
@@ -62,16 +69,18 @@ cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes,
   cudaError_t err = cudaFuncSetAttribute(hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  err = cudaFuncSetAttribute(scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  err = cudaFuncSetAttribute(slots_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
   if (err != cudaSuccess) return err;
-  count_launch(4);
+  count_launch(5);
   hist_kernel<<<blocks, 32 * kWarps, smem, s>>>(topk_idx, T, E, k, C, cnt);
   scan_kernel<<<(E + 31) / 32, 1024, 0, s>>>(cnt, E, C, totals);
   offsets_kernel<<<1, 1024, 0, s>>>(totals, E, offsets);
-  scatter_kernel<<<blocks, 32 * kWarps, smem, s>>>(
-      static_cast<const uint8_t*>(x), x_scales, row_bytes, H / 128, topk_idx, T, E, k, C, cnt,
-      offsets, static_cast<uint8_t*>(x_perm), x_perm_scales, perm_src, slot_of);
+  slots_kernel<<<blocks, 32 * kWarps, smem, s>>>(topk_idx, T, E, k, C, cnt, offsets, perm_src,
+                                                 slot_of);
+  copy_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(static_cast<const uint8_t*>(x), x_scales,
+                                               row_bytes, H / 128, slot_of, T, k,
+                                               static_cast<uint8_t*>(x_perm), x_perm_scales);
   return cudaGetLastError();
 }
 

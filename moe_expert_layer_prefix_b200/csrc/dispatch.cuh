@@ -13,8 +13,8 @@
 //   slot(t, j) = offsets[e] + (tokens of e in earlier chunks) + popc(mask_e & below(t)).
 //
 // Steps: hist (per-chunk counts) -> scan (per-expert exclusive scan over chunks, totals)
-// -> offsets (exclusive scan over experts) -> scatter (slots, permutation, row copies).
-// The row copy reads each x row once and writes it k times with 16-byte accesses.
+// -> offsets (exclusive scan over experts) -> slots (permutation) -> row copies (one warp
+// per token, each x row read once and written k times with 16-byte accesses).
 // These device functions are shared by the dispatch kernels and the persistent forward
 // kernel.
 #pragma once
@@ -120,16 +120,15 @@ __device__ __forceinline__ void offsets_from_totals(const int32_t* totals, int E
   __syncthreads();
 }
 
-// Slots, permutation and row copies of one 32-token chunk (one warp).  mask: E words of
-// shared memory; sslot: shared [32][32]; bases: chunk bases from scan_group; offsets:
-// expert offsets (global or shared).
-__device__ __forceinline__ void scatter_chunk(
-    uint32_t* mask, int32_t (*sslot)[32], const uint8_t* __restrict__ x,
-    const float* __restrict__ x_scales, int row_bytes, int nscale,
-    const int32_t* __restrict__ topk_idx, int T, int E, int k, int chunk,
-    const int32_t* __restrict__ bases, const int32_t* offsets, uint8_t* __restrict__ x_perm,
-    float* __restrict__ x_perm_scales, int32_t* __restrict__ perm_src,
-    int32_t* __restrict__ slot_of, int lane) {
+// Slots and permutation of one 32-token chunk (one warp).  mask: E words of shared memory;
+// bases: chunk bases from scan_group; offsets: expert offsets (global or shared).
+__device__ __forceinline__ void assign_slots_chunk(uint32_t* mask,
+                                                   const int32_t* __restrict__ topk_idx, int T,
+                                                   int E, int k, int chunk,
+                                                   const int32_t* __restrict__ bases,
+                                                   const int32_t* offsets,
+                                                   int32_t* __restrict__ perm_src,
+                                                   int32_t* __restrict__ slot_of, int lane) {
   build_chunk_mask(mask, topk_idx, T, E, k, chunk, lane);
   const int t = chunk * kChunkTokens + lane;
   if (t < T) {
@@ -141,32 +140,51 @@ __device__ __forceinline__ void scatter_chunk(
       const int src = t * k + j;
       slot_of[src] = slot;
       perm_src[slot] = src;
-      sslot[lane][j] = slot;
     }
   }
   __syncwarp();
-  // the warp walks its chunk's tokens; each 16-byte piece of a row is loaded once and stored
-  // to the token's k slots
-  const int ntok = min(kChunkTokens, T - chunk * kChunkTokens);
+}
+
+// Row copies of token t (one warp): its row of x (and of x_scales) goes to its k slots.
+// Each 16-byte piece is read once; a lane keeps up to kV pieces in flight.
+__device__ __forceinline__ void copy_token_rows(const uint8_t* __restrict__ x,
+                                                const float* __restrict__ x_scales,
+                                                int row_bytes, int nscale,
+                                                const int32_t* __restrict__ slot_of, int t, int k,
+                                                uint8_t* __restrict__ x_perm,
+                                                float* __restrict__ x_perm_scales, int lane) {
+  constexpr int kV = 8;
+  int my_slot = 0;
+  if (lane < k) my_slot = __ldcg(slot_of + static_cast<size_t>(t) * k + lane);
+  int slots[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) slots[j] = __shfl_sync(0xffffffffu, my_slot, j);
   const int nvec = row_bytes / 16;
-  for (int i = 0; i < ntok; ++i) {
-    const int tt = chunk * kChunkTokens + i;
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(tt) * row_bytes);
-    for (int v = lane; v < nvec; v += 32) {
-      const uint4 d = __ldg(src + v);
-      for (int j = 0; j < k; ++j) {
-        uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(sslot[i][j]) * row_bytes);
-        dst[v] = d;
-      }
+  const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * row_bytes);
+  for (int v0 = lane; v0 < nvec; v0 += 32 * kV) {
+    uint4 d[kV];
+#pragma unroll
+    for (int u = 0; u < kV; ++u)
+      if (v0 + 32 * u < nvec) d[u] = __ldg(src + v0 + 32 * u);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (j >= k) break;
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + static_cast<size_t>(slots[j]) * row_bytes);
+#pragma unroll
+      for (int u = 0; u < kV; ++u)
+        if (v0 + 32 * u < nvec) dst[v0 + 32 * u] = d[u];
     }
-    if (x_scales != nullptr) {
-      for (int v = lane; v < nscale; v += 32) {
-        const float sv = __ldg(x_scales + static_cast<size_t>(tt) * nscale + v);
-        for (int j = 0; j < k; ++j) x_perm_scales[static_cast<size_t>(sslot[i][j]) * nscale + v] = sv;
+  }
+  if (x_scales != nullptr) {
+    for (int v = lane; v < nscale; v += 32) {
+      const float sv = __ldg(x_scales + static_cast<size_t>(t) * nscale + v);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= k) break;
+        x_perm_scales[static_cast<size_t>(slots[j]) * nscale + v] = sv;
       }
     }
   }
-  __syncwarp();
 }
 
 }  // namespace moe

@@ -75,14 +75,18 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   // dispatch scratch inside the (idle) GEMM ring: per-warp chunk masks in the A stages,
   // slot tables, scan partials and offsets in the B stages
   uint32_t* mask = reinterpret_cast<uint32_t*>(sm.sA) + warp * p.E;
-  int32_t(*sslot)[32] = reinterpret_cast<int32_t(*)[32]>(sm.sB) + warp * kChunkTokens;
   int32_t(*part)[33] = reinterpret_cast<int32_t(*)[33]>(sm.sB + nwarps * kChunkTokens * 32 * 4);
   int32_t* soffs = reinterpret_cast<int32_t*>(sm.sB + nwarps * kChunkTokens * 32 * 4 + 32 * 33 * 4);
   int32_t* wsum = soffs + 1028;
 
   // 1. route: one warp per token
-  for (int t = gw; t < p.T; t += GW)
-    route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+  if (p.E <= 256) {
+    for (int t = gw; t < p.T; t += GW)
+      route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+  } else {
+    for (int t = gw; t < p.T; t += GW)
+      route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+  }
   grid_sync(p.bar, p.err);
 
   // 2. per-chunk expert counts
@@ -99,15 +103,20 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   if (blockIdx.x == 0)
     for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.offsets[e] = soffs[e];
 
-  // 5. slots, permutation and row copies
+  // 5. slots and permutation (one warp per 32-token chunk)
   for (int c = gw; c < p.C; c += GW)
-    scatter_chunk(mask, sslot, static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes,
-                  p.H / 128, p.topk_idx, p.T, p.E, p.k, c, p.cnt, soffs,
-                  static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, p.perm_src, p.slot_of, lane);
+    assign_slots_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, p.cnt, soffs, p.perm_src, p.slot_of,
+                       lane);
+  grid_sync(p.bar, p.err);
+
+  // 6. row copies x -> x_perm (one warp per token)
+  for (int t = gw; t < p.T; t += GW)
+    copy_token_rows(static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes, p.H / 128,
+                    p.slot_of, t, p.k, static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
   fence_proxy_async_global();  // x_perm is read by TMA next
   grid_sync(p.bar, p.err);
 
-  // 6. linear-1 + SwiGLU + requantisation
+  // 7. linear-1 + SwiGLU + requantisation
   Pipe pipe;
   gemm_prefix<1>(sm, p.offsets, p.E, p.l1.n_tiles);
   tc_fence_before();
@@ -117,7 +126,7 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   fence_proxy_async_global();  // h is read by TMA next
   grid_sync(p.bar, p.err);
 
-  // 7. linear-2
+  // 8. linear-2
   gemm_prefix<1>(sm, p.offsets, p.E, p.l2.n_tiles);
   tc_fence_before();
   __syncthreads();
@@ -125,9 +134,9 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   gemm_phase<1, kBS, kBFmt, false, false>(&tmH, &tmW2, p.l2, sm, pipe);
   grid_sync(p.bar, p.err);
 
-  // 8. combine: one warp per token
+  // 9. combine: one warp per token
   for (int t = gw; t < p.T; t += GW)
-    combine_token(p.y, 0, p.slot_of, p.topk_w, t, p.k, p.H, p.out, 0, lane);
+    combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane);
 
   tc_fence_before();
   __syncthreads();
