@@ -67,8 +67,8 @@ constexpr int kSfSets = 4;         // rotated per k-step so a copy never waits o
 constexpr int kThreads = 256;
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
-constexpr int kRawWords = 12;       // raw scale words per lane per k-step (4 A + up to 8 B)
-constexpr int kRawBytes = 32 * kRawWords * 4;
+constexpr int kSfSlots = 16;       // scale-factor ring, decoupled from (and deeper than) the A/B ring
+constexpr int kSfBatch = 8;        // slots the converter publishes with one warp-wide arrive
 
 struct TcParams {
   const int32_t* offsets;  // [E+1]
@@ -87,8 +87,9 @@ struct TcParams {
 struct SharedState {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t raw_full[kMaxStages];   // scale words staged by the loader warp
-  uint64_t raw_empty[kMaxStages];  // ... and consumed by the converter warp
+  uint64_t sf_raw[kSfSlots];    // loader -> converter: raw scale words staged in the slot
+  uint64_t sf_full[kSfSlots];   // converters -> MMA issuer: slot converted (one per CTA)
+  uint64_t sf_empty[kSfSlots];  // MMA issuer -> loaders: slot copied to TMEM and consumed
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
@@ -106,8 +107,8 @@ struct Cfg {
   static constexpr int kBTileBytes = kBRows * kRowBytes;  // 32 KB single, 16 KB pair
   static constexpr int kTileM = kBM * kCta;               // rows of one tile
   static constexpr size_t kSmem = 1024 + kStages * (kATileBytes + kBTileBytes) +
-                                  kStages * (kSfaBytes + kSfbBytes) + kStages * kRawBytes +
-                                  sizeof(SharedState);
+                                  kSfSlots * (kSfaBytes + kSfbBytes) + sizeof(SharedState);
+  static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
 
 struct Tile {
@@ -150,7 +151,6 @@ struct Smem {
   uint8_t* sA;
   uint8_t* sB;
   uint8_t* sSF;
-  uint8_t* sRaw;
   SharedState* ss;
 };
 
@@ -161,9 +161,8 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw) {
   m.sA = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                     ~static_cast<uintptr_t>(1023));
   m.sB = m.sA + C::kStages * kATileBytes;
-  m.sSF = m.sB + C::kStages * C::kBTileBytes;             // per stage: SFA 512 B, SFB 1024 B
-  m.sRaw = m.sSF + C::kStages * (kSfaBytes + kSfbBytes);  // per stage: [lane][kRawWords]
-  m.ss = reinterpret_cast<SharedState*>(m.sRaw + C::kStages * kRawBytes);
+  m.sSF = m.sB + C::kStages * C::kBTileBytes;             // per slot: SFA 512 B, SFB 1024 B
+  m.ss = reinterpret_cast<SharedState*>(m.sSF + kSfSlots * (kSfaBytes + kSfbBytes));
   return m;
 }
 
@@ -175,10 +174,13 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < Cfg<kCta>::kStages; ++s) {
-      mbar_init(&ss.full[s], 1 + (kBlockScaled ? kCta : 0));
+      mbar_init(&ss.full[s], 1);
       mbar_init(&ss.empty[s], 1);
-      mbar_init(&ss.raw_full[s], 1);
-      mbar_init(&ss.raw_empty[s], 1);
+    }
+    for (int s = 0; s < kSfSlots; ++s) {
+      mbar_init(&ss.sf_raw[s], 32);  // one cp.async completion arrival per loader lane
+      mbar_init(&ss.sf_full[s], kCta);
+      mbar_init(&ss.sf_empty[s], 1);
     }
     mbar_init(&ss.acc_full, 1);
     mbar_init(&ss.acc_empty, 4 * kCta);
@@ -253,7 +255,6 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
   uint8_t* sA = sm.sA;
   uint8_t* sB = sm.sB;
   uint8_t* sSF = sm.sSF;
-  uint8_t* sRaw = sm.sRaw;
   SharedState& ss = *sm.ss;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
@@ -340,6 +341,14 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             ok = false;
             break;
           }
+          const int slot = static_cast<int>(it % kSfSlots);
+          if constexpr (kBlockScaled) {
+            if (!mbar_wait<kPair>(&ss.sf_full[slot], (it / kSfSlots) & 1u, p.err, SITE_GEMM_FULL,
+                                  abort)) {
+              ok = false;
+              break;
+            }
+          }
           tc_fence_after();
           const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * kATileBytes));
           const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
@@ -347,7 +356,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           const uint32_t tsfa = tmem + kSfaCol + sfset * kSfSetCols;
           const uint32_t tsfb = tmem + kSfbCol + sfset * kSfSetCols;
           if constexpr (kBlockScaled) {
-            const uint32_t sf = smem_u32(sSF + stage * (kSfaBytes + kSfbBytes));
+            const uint32_t sf = smem_u32(sSF + slot * (kSfaBytes + kSfbBytes));
             if constexpr (kPair) {
               tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sf));
               tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sf + kSfaBytes));
@@ -379,6 +388,10 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           issued_any = true;
           if constexpr (kPair) tc_commit_pair(&ss.empty[stage], 0x3);
           else tc_commit(&ss.empty[stage]);
+          if constexpr (kBlockScaled) {
+            if constexpr (kPair) tc_commit_pair(&ss.sf_empty[slot], 0x3);
+            else tc_commit(&ss.sf_empty[slot]);
+          }
           ++it;
         }
         if (!ok) break;
@@ -400,22 +413,23 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------------ scale loader
-    // Iterations i = (tile, k-step) of this CTA in order.  The raw scale words of iteration
-    // i + kSfDepth are loaded right after iteration i is staged, so their latency overlaps
-    // kSfDepth k-steps; row pointers are set up once per tile.  Words are staged in a small
-    // shared-memory ring for the converter warp, which therefore never has global loads in
-    // flight when it signals the (pair leader's) stage barrier.
+    // Iterations i = (tile, k-step) of this CTA in order; iteration i uses scale slot
+    // i % kSfSlots.  Each lane copies the raw scale words of its rows straight into the slot
+    // at their final positions with asynchronous 4-byte copies whose completion arrives on the
+    // slot's raw barrier, so the loader runs up to kSfSlots k-steps ahead of the MMA issuer
+    // with nothing held in registers; row pointers are set up once per tile.  Each CTA copies
+    // the scales of its own A rows and of all 256 B rows of the tile; the converter warp then
+    // rewrites the slot in place.
     if constexpr (kBlockScaled) {
-      constexpr int kSfDepth = 4;
       constexpr int kNB = kBFmt == 5 ? 8 : 2;  // B words per lane per k-step
       const int KS = p.K / 128;                // fp32 scale columns of A (and of E4M3 B)
-      uint32_t ra[kSfDepth][4];
-      uint32_t rb[kSfDepth][kNB];
-      int lt = cid, lkb = 0;  // loader state: the next (tile, k-step) to load
       const float* pa[4];
       const uint8_t* pb[kNB];
-      auto setup_tile = [&]() {
-        if (lt >= total) return;
+      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
+      const uint32_t it0 = pipe.sf_it;
+      uint32_t gi = it0;
+      bool ok = true;
+      for (int lt = cid; lt < total && ok; lt += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1) {
@@ -445,105 +459,79 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
                 (static_cast<size_t>(tile.e) * (p.w_rows / 128) + wr / 128) * KS);
           }
         }
-      };
-      auto load_next = [&](uint32_t (&a4)[4], uint32_t (&bw)[kNB]) {
-        if (lt >= total) return;
-#pragma unroll
-        for (int r1 = 0; r1 < 4; ++r1) a4[r1] = __float_as_uint(__ldcg(pa[r1] + lkb));
-        if constexpr (kBFmt == 5) {
-#pragma unroll
-          for (int r = 0; r < 8; ++r) bw[r] = __ldg(reinterpret_cast<const uint32_t*>(pb[r] + lkb * 4));
-        } else {
-#pragma unroll
-          for (int a = 0; a < 2; ++a)
-            bw[a] = __float_as_uint(__ldg(reinterpret_cast<const float*>(pb[a]) + lkb));
-        }
-        if (++lkb == KB) {
-          lkb = 0;
-          lt += ncl;
-          setup_tile();
-        }
-      };
-      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
-      const int n_iter = my_tiles * KB;
-      setup_tile();
-#pragma unroll
-      for (int j = 0; j < kSfDepth; ++j) load_next(ra[j], rb[j]);
-      bool ok = true;
-      const uint32_t it0 = pipe.sf_it;
-      for (int base = 0; base < n_iter && ok; base += kSfDepth) {
-#pragma unroll
-        for (int j = 0; j < kSfDepth; ++j) {
-          const int i = base + j;
-          if (i >= n_iter) break;
-          const int stage = static_cast<int>((it0 + i) % kStages);
-          const uint32_t phase = ((it0 + i) / kStages) & 1u;
-          if (!mbar_wait(&ss.raw_empty[stage], phase ^ 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) {
+        for (int kb = 0; kb < KB; ++kb, ++gi) {
+          const int slot = static_cast<int>(gi % kSfSlots);
+          if (!mbar_wait<kPair>(&ss.sf_empty[slot], ((gi / kSfSlots) & 1u) ^ 1u, p.err,
+                                SITE_GEMM_SF_EMPTY, abort)) {
             ok = false;
             break;
           }
-          uint32_t* raw = reinterpret_cast<uint32_t*>(sRaw + stage * kRawBytes) + lane * kRawWords;
-          *reinterpret_cast<uint4*>(raw) = make_uint4(ra[j][0], ra[j][1], ra[j][2], ra[j][3]);
+          uint8_t* sf = sSF + slot * (kSfaBytes + kSfbBytes);
+#pragma unroll
+          for (int r1 = 0; r1 < 4; ++r1) cp_async_4(sf + 16 * lane + 4 * r1, pa[r1] + kb);
           if constexpr (kBFmt == 5) {
-            *reinterpret_cast<uint4*>(raw + 4) = make_uint4(rb[j][0], rb[j][1], rb[j][2], rb[j][3]);
-            *reinterpret_cast<uint4*>(raw + 8) = make_uint4(rb[j][4], rb[j][5], rb[j][6], rb[j][7]);
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              cp_async_4(sf + kSfaBytes + 512 * (r >> 2) + 16 * lane + 4 * (r & 3), pb[r] + 4 * kb);
           } else {
-            *reinterpret_cast<uint2*>(raw + 4) = make_uint2(rb[j][0], rb[j][1]);
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+              cp_async_4(sf + kSfaBytes + 16 * lane + 4 * a,
+                         reinterpret_cast<const float*>(pb[a]) + kb);
           }
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ss.raw_full[stage]);
-          load_next(ra[j], rb[j]);
+          cp_async_mbar_arrive(&ss.sf_raw[slot]);
         }
       }
-      pipe.sf_it = it0 + n_iter;
+      cp_async_wait_all();  // no copy may still be landing when the CTA moves on
+      pipe.sf_it = it0 + static_cast<uint32_t>(my_tiles * KB);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------------ scale converter
-    // Turns the staged fp32 / UE8M0 words into the shared-memory layout tcgen05.cp reads
-    // (32 rows x 16 bytes per 128-row atom: byte 16*(r%32) + 4*(r/32) + k-sub-block) and
-    // signals the stage barrier of the pair leader.
+    // Rewrites each staged slot in place into the layout tcgen05.cp reads (32 rows x 16
+    // bytes per 128-row atom: byte 16*(r%32) + 4*(r/32) + k-sub-block; fp32 power-of-two
+    // scales become their UE8M0 exponent byte, x4 along K) and publishes kSfBatch slots at
+    // a time with one warp-wide arrive on the (pair leader's) slot barriers, so the
+    // cluster-scope release that makes the slots visible is paid once per batch.
     if constexpr (kBlockScaled) {
       const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
       const int n_iter = my_tiles * KB;
-      const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.full[0]), 0);
       const uint32_t it0 = pipe.sf_it;
-      for (int i = 0; i < n_iter; ++i) {
-        const int stage = static_cast<int>((it0 + i) % kStages);
-        const uint32_t phase = ((it0 + i) / kStages) & 1u;
-        if (!mbar_wait(&ss.raw_full[stage], phase, p.err, SITE_GEMM_SF_EMPTY, abort)) break;
-        if (!mbar_wait<kPair>(&ss.empty[stage], phase ^ 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) break;
-        const uint32_t* raw = reinterpret_cast<const uint32_t*>(sRaw + stage * kRawBytes) + lane * kRawWords;
-        const uint4 ra4 = *reinterpret_cast<const uint4*>(raw);
-        uint32_t b8[8];
-        if constexpr (kBFmt == 5) {
-          const uint4 lo = *reinterpret_cast<const uint4*>(raw + 4);
-          const uint4 hi = *reinterpret_cast<const uint4*>(raw + 8);
-          b8[0] = lo.x; b8[1] = lo.y; b8[2] = lo.z; b8[3] = lo.w;
-          b8[4] = hi.x; b8[5] = hi.y; b8[6] = hi.z; b8[7] = hi.w;
-        } else {
-          const uint2 w2 = *reinterpret_cast<const uint2*>(raw + 4);
-          const uint32_t v0 = ((w2.x >> 23) & 0xFFu) * 0x01010101u;
-          const uint32_t v1 = ((w2.y >> 23) & 0xFFu) * 0x01010101u;
-          b8[0] = b8[1] = b8[2] = b8[3] = v0;
-          b8[4] = b8[5] = b8[6] = b8[7] = v1;
+      const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
+      bool ok = true;
+      for (int b = 0; b < n_iter && ok; b += kSfBatch) {
+        const int cnt = n_iter - b < kSfBatch ? n_iter - b : kSfBatch;
+        for (int j = 0; j < cnt; ++j) {
+          const uint32_t gi = it0 + static_cast<uint32_t>(b + j);
+          const int slot = static_cast<int>(gi % kSfSlots);
+          if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfSlots) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sf = sSF + slot * (kSfaBytes + kSfbBytes);
+          const uint4 a = *reinterpret_cast<const uint4*>(sf + 16 * lane);
+          *reinterpret_cast<uint4*>(sf + 16 * lane) =
+              make_uint4(((a.x >> 23) & 0xFFu) * 0x01010101u, ((a.y >> 23) & 0xFFu) * 0x01010101u,
+                         ((a.z >> 23) & 0xFFu) * 0x01010101u, ((a.w >> 23) & 0xFFu) * 0x01010101u);
+          if constexpr (kBFmt == 5) {
+            // already UE8M0 bytes in atom order; rewritten so that this warp's proxy fence
+            // covers every byte tcgen05.cp reads, not only the converted ones
+            smem_touch16(sf + kSfaBytes + 16 * lane);
+            smem_touch16(sf + kSfaBytes + 512 + 16 * lane);
+          } else {
+            const uint2 w2 = *reinterpret_cast<const uint2*>(sf + kSfaBytes + 16 * lane);
+            const uint32_t v0 = ((w2.x >> 23) & 0xFFu) * 0x01010101u;
+            const uint32_t v1 = ((w2.y >> 23) & 0xFFu) * 0x01010101u;
+            *reinterpret_cast<uint4*>(sf + kSfaBytes + 16 * lane) = make_uint4(v0, v0, v0, v0);
+            *reinterpret_cast<uint4*>(sf + kSfaBytes + 512 + 16 * lane) = make_uint4(v1, v1, v1, v1);
+          }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ss.raw_empty[stage]);
-        // fp32 power-of-two scale -> its UE8M0 byte (the biased exponent), x4 along K
-        const uint32_t a0 = ((ra4.x >> 23) & 0xFFu) * 0x01010101u;
-        const uint32_t a1 = ((ra4.y >> 23) & 0xFFu) * 0x01010101u;
-        const uint32_t a2 = ((ra4.z >> 23) & 0xFFu) * 0x01010101u;
-        const uint32_t a3 = ((ra4.w >> 23) & 0xFFu) * 0x01010101u;
-        uint8_t* sf = sSF + stage * (kSfaBytes + kSfbBytes);
-        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(a0, a1, a2, a3);
-        *reinterpret_cast<uint4*>(sf + kSfaBytes + 16 * lane) = make_uint4(b8[0], b8[1], b8[2], b8[3]);
-        *reinterpret_cast<uint4*>(sf + kSfaBytes + 512 + 16 * lane) =
-            make_uint4(b8[4], b8[5], b8[6], b8[7]);
+        if (!ok) break;
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(full_lead0 + stage * sizeof(uint64_t));
-          else mbar_arrive(&ss.full[stage]);
+        if (lane < cnt) {
+          const int slot = static_cast<int>((it0 + static_cast<uint32_t>(b + lane)) % kSfSlots);
+          if constexpr (kPair) mbar_arrive_cluster(full_lead0 + slot * sizeof(uint64_t));
+          else mbar_arrive(&ss.sf_full[slot]);
         }
       }
       pipe.sf_it = it0 + n_iter;
