@@ -144,6 +144,7 @@ struct Pipe {
   uint32_t mma_it = 0;   // MMA issuer: k-steps consumed
   uint32_t tiles = 0;    // MMA issuer / epilogue: accumulator uses
   uint32_t sf_it = 0;    // scale loader / converter: k-steps staged
+  uint32_t sf_grp = 0;   // MMA issuer: groups of 4 k-steps whose scales were copied to TMEM
 };
 
 // Shared-memory carve-up (1024-byte aligned; identical offsets in both CTAs of a pair).
@@ -326,7 +327,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       constexpr int kMmaM = kBM * kCta;
       constexpr uint32_t kIdesc = kBlockScaled ? idesc_mxf8f6f4(kMmaM, kBN, 0u, kBFmt)
                                                : idesc_bf16(kMmaM, kBN);
-      uint32_t it = pipe.mma_it, tiles = pipe.tiles;
+      uint32_t it = pipe.mma_it, tiles = pipe.tiles, grp = pipe.sf_grp;
       bool issued_any = false;
       for (int t = cid; t < total && !*abort; t += ncl) {
         const uint32_t acc_phase = tiles & 1u;
@@ -342,29 +343,43 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             break;
           }
           const int slot = static_cast<int>(it % kSfSlots);
+          const bool grp_start = (kb & 3) == 0;
           if constexpr (kBlockScaled) {
-            if (!mbar_wait<kPair>(&ss.sf_full[slot], (it / kSfSlots) & 1u, p.err, SITE_GEMM_FULL,
-                                  abort)) {
-              ok = false;
-              break;
+            // the scales of a group of 4 k-steps are published together; slots are converted
+            // and published in order, so the group's last slot covers the whole group
+            if (grp_start) {
+              const uint32_t il = it + static_cast<uint32_t>(min(kb + 3, KB - 1) - kb);
+              if (!mbar_wait<kPair>(&ss.sf_full[il % kSfSlots], (il / kSfSlots) & 1u, p.err,
+                                    SITE_GEMM_FULL, abort)) {
+                ok = false;
+                break;
+              }
             }
           }
           tc_fence_after();
           const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * kATileBytes));
           const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
-          const uint32_t sfset = it % kSfSets;
-          const uint32_t tsfa = tmem + kSfaCol + sfset * kSfSetCols;
-          const uint32_t tsfb = tmem + kSfbCol + sfset * kSfSetCols;
+          if (grp_start) ++grp;
+          // A scales (and E4M3 B scales) are per 128 of K, so one byte per k-step: a group of
+          // 4 k-steps shares one copy, byte kb % 4 selecting the k-step.  E2M1 B scales are per
+          // 32 of K (byte = sub-block) and are copied every k-step.
+          const uint32_t tsfa = tmem + kSfaCol + (grp % kSfSets) * kSfSetCols;
+          const uint32_t tsfb =
+              tmem + kSfbCol + (kBFmt == 5 ? it % kSfSets : grp % kSfSets) * kSfSetCols;
           if constexpr (kBlockScaled) {
             const uint32_t sf = smem_u32(sSF + slot * (kSfaBytes + kSfbBytes));
-            if constexpr (kPair) {
-              tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sf));
-              tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sf + kSfaBytes));
-              tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
-            } else {
-              tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sf));
-              tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sf + kSfaBytes));
-              tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+            if (grp_start) {
+              if constexpr (kPair) tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sf));
+              else tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sf));
+            }
+            if (kBFmt == 5 || grp_start) {
+              if constexpr (kPair) {
+                tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sf + kSfaBytes));
+                tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+              } else {
+                tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sf + kSfaBytes));
+                tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+              }
             }
           }
 #pragma unroll
@@ -374,10 +389,11 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             const uint64_t bd = bdesc + static_cast<uint64_t>(ks * 2);
             const uint32_t acc = (kb | ks) != 0 ? 1u : 0u;
             if constexpr (kBlockScaled) {
-              const uint32_t id = kIdesc | (static_cast<uint32_t>(ks) << 4) |
-                                  (static_cast<uint32_t>(ks) << 29);
-              const uint32_t sfa = tsfa | (static_cast<uint32_t>(ks) << 30);
-              const uint32_t sfb = tsfb | (static_cast<uint32_t>(ks) << 30);
+              const uint32_t a_id = static_cast<uint32_t>(kb & 3);
+              const uint32_t b_id = kBFmt == 5 ? static_cast<uint32_t>(ks) : a_id;
+              const uint32_t id = kIdesc | (b_id << 4) | (a_id << 29);
+              const uint32_t sfa = tsfa | (a_id << 30);
+              const uint32_t sfb = tsfb | (b_id << 30);
               if constexpr (kPair) mma_mxf8f6f4_pair(tmem + kAccCol, ad, bd, id, sfa, sfb, acc);
               else mma_mxf8f6f4(tmem + kAccCol, ad, bd, id, sfa, sfb, acc);
             } else {
@@ -401,6 +417,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       }
       pipe.mma_it = it;
       pipe.tiles = tiles;
+      pipe.sf_grp = grp;
       if (*abort && issued_any) {
         // let the issued MMAs finish before TMEM is released
         if constexpr (kPair) tc_commit_pair(&ss.drain, 0x1);
@@ -487,11 +504,17 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------------ scale converter
-    // Rewrites each staged slot in place into the layout tcgen05.cp reads (32 rows x 16
-    // bytes per 128-row atom: byte 16*(r%32) + 4*(r/32) + k-sub-block; fp32 power-of-two
-    // scales become their UE8M0 exponent byte, x4 along K) and publishes kSfBatch slots at
-    // a time with one warp-wide arrive on the (pair leader's) slot barriers, so the
-    // cluster-scope release that makes the slots visible is paid once per batch.
+    // Rewrites the staged raw words into the layout tcgen05.cp reads: per 128-row atom, 32
+    // lines of 16 bytes, byte 16*(r%32) + 4*(r/32) + b for row r, one UE8M0 (the exponent
+    // byte of a power-of-two fp32 scale) per byte.  A scales and E4M3 B scales cover 128 of K,
+    // so b indexes the k-step inside a group of 4 k-steps of a tile: once the group's last
+    // k-step is staged, its packed atoms are written into the slot of the group's first
+    // k-step (one TMEM copy per group).  E2M1 B scales are per 32 of K and already UE8M0 in
+    // atom order (b = sub-block).  kSfBatch slots are published at a time with one warp-wide
+    // arrive on the (pair leader's) slot barriers, so the cluster-scope release that makes
+    // them visible is paid once per batch; kSfBatch + 4 <= kSfSlots keeps the loader free to
+    // stage every slot a published group needs.
+    static_assert(kSfBatch + 4 <= kSfSlots, "scale ring too shallow for batch + group");
     if constexpr (kBlockScaled) {
       const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
       const int n_iter = my_tiles * KB;
@@ -508,21 +531,37 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             break;
           }
           uint8_t* sf = sSF + slot * (kSfaBytes + kSfbBytes);
-          const uint4 a = *reinterpret_cast<const uint4*>(sf + 16 * lane);
-          *reinterpret_cast<uint4*>(sf + 16 * lane) =
-              make_uint4(((a.x >> 23) & 0xFFu) * 0x01010101u, ((a.y >> 23) & 0xFFu) * 0x01010101u,
-                         ((a.z >> 23) & 0xFFu) * 0x01010101u, ((a.w >> 23) & 0xFFu) * 0x01010101u);
           if constexpr (kBFmt == 5) {
-            // already UE8M0 bytes in atom order; rewritten so that this warp's proxy fence
-            // covers every byte tcgen05.cp reads, not only the converted ones
+            // rewritten so that this warp's proxy fence covers every byte tcgen05.cp reads
             smem_touch16(sf + kSfaBytes + 16 * lane);
             smem_touch16(sf + kSfaBytes + 512 + 16 * lane);
-          } else {
-            const uint2 w2 = *reinterpret_cast<const uint2*>(sf + kSfaBytes + 16 * lane);
-            const uint32_t v0 = ((w2.x >> 23) & 0xFFu) * 0x01010101u;
-            const uint32_t v1 = ((w2.y >> 23) & 0xFFu) * 0x01010101u;
-            *reinterpret_cast<uint4*>(sf + kSfaBytes + 16 * lane) = make_uint4(v0, v0, v0, v0);
-            *reinterpret_cast<uint4*>(sf + kSfaBytes + 512 + 16 * lane) = make_uint4(v1, v1, v1, v1);
+          }
+          const int kb = (b + j) % KB;
+          const int g0 = kb & ~3;
+          if (kb == KB - 1 || (kb & 3) == 3) {
+            uint32_t wa0 = 0, wa1 = 0, wa2 = 0, wa3 = 0, wb0 = 0, wb1 = 0;
+            for (int q = 0; q <= kb - g0; ++q) {
+              const uint8_t* src =
+                  sSF + ((gi - static_cast<uint32_t>(kb - g0 - q)) % kSfSlots) * (kSfaBytes + kSfbBytes);
+              const uint4 a = *reinterpret_cast<const uint4*>(src + 16 * lane);
+              wa0 |= ((a.x >> 23) & 0xFFu) << (8 * q);
+              wa1 |= ((a.y >> 23) & 0xFFu) << (8 * q);
+              wa2 |= ((a.z >> 23) & 0xFFu) << (8 * q);
+              wa3 |= ((a.w >> 23) & 0xFFu) << (8 * q);
+              if constexpr (kBFmt != 5) {
+                const uint2 w2 = *reinterpret_cast<const uint2*>(src + kSfaBytes + 16 * lane);
+                wb0 |= ((w2.x >> 23) & 0xFFu) << (8 * q);
+                wb1 |= ((w2.y >> 23) & 0xFFu) << (8 * q);
+              }
+            }
+            uint8_t* dst =
+                sSF + ((gi - static_cast<uint32_t>(kb - g0)) % kSfSlots) * (kSfaBytes + kSfbBytes);
+            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(wa0, wa1, wa2, wa3);
+            if constexpr (kBFmt != 5) {
+              *reinterpret_cast<uint4*>(dst + kSfaBytes + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
+              *reinterpret_cast<uint4*>(dst + kSfaBytes + 512 + 16 * lane) =
+                  make_uint4(wb1, wb1, wb1, wb1);
+            }
           }
         }
         if (!ok) break;
