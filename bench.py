@@ -314,10 +314,15 @@ def run_native(args, ws, rank, local):
                if (alg[dom]["flops"] and tens_mult) else 0.0)
     t_bytes = alg[dom]["bytes"] / (pk["hbm_gbs"] * 1e9)
     if t_flops >= t_bytes and alg[dom]["flops"]:
+        # the GEMM is timed inside a loop of back-to-back steps, where the power cap holds
+        # the clock well below its maximum: the sustained figure is the matching peak
+        sus = "bf16_tflops_sustained" in pk
+        peak_bf16 = pk["bf16_tflops_sustained"] if sus else pk["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": alg[dom]["flops"] / dsec / 1e12,
-                "peak": pk["bf16_tflops"] * tens_mult, "unit": "TFLOP/s"}
-        roof["peak_note"] = (f"{pk_kind} bf16 burst x {tens_mult:g} (nominal "
-                             f"{'fp8' if tens_mult == 2 else 'bf16'}:bf16 ratio)")
+                "peak": peak_bf16 * tens_mult, "unit": "TFLOP/s"}
+        roof["peak_note"] = (f"{pk_kind} bf16 {'sustained' if sus else 'burst'} x {tens_mult:g} "
+                             f"(nominal {'fp8' if tens_mult == 2 else 'bf16'}:bf16 ratio)")
+        roof["frac_of_burst"] = roof["achieved"] / (pk["bf16_tflops"] * tens_mult)
     else:
         roof = {"bound": "hbm", "achieved": alg[dom]["bytes"] / dsec / 1e9,
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_note": f"{pk_kind} copy bandwidth"}
@@ -442,7 +447,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="v3_fp8", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair"],
+    ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair", "small"],
                     help="tile shape of the expert GEMMs")
     ap.add_argument("--T", type=int, default=None, help="override T (profiling captures)")
     ap.add_argument("--E", type=int, default=None, help="override E (profiling captures)")

@@ -202,9 +202,12 @@ const char* moe_status_string(int status);
 uint64_t moe_launch_count(void);
 
 /* Process-wide tile shape of the tensor-core expert GEMMs (a tuning and testing knob):
- * 0 automatic (CTA pairs, M = 256 per tile, when S >= 128 * E; single CTAs, M = 128,
- * otherwise), 1 always single CTAs, 2 always CTA pairs.  Results are identical up to fp32
- * accumulation order.  Returns MOE_ERR_INVALID_ARG for any other value. */
+ * 0 automatic, 1 always single CTAs (128-row tiles), 2 always CTA pairs (256-row tiles on
+ * cta_group::2; moe_forward's single launch uses single CTAs instead), 3 always small tiles
+ * (32-row m-blocks, one CTA).  Automatic: small tiles when S <= 16 * E (decode-sized
+ * batches), pairs for BF16 when S >= 128 * E, single CTAs otherwise.  Single and small tiles
+ * give identical bits; pairs are identical up to fp32 accumulation order.  Returns
+ * MOE_ERR_INVALID_ARG for any other value. */
 moe_status moe_set_gemm_tiles(int mode);
 
 #ifdef __cplusplus

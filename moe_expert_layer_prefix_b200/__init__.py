@@ -85,12 +85,12 @@ def moe_launch_count() -> int:
     return int(_launch_count())
 
 
-TILES = {"auto": 0, "single": 1, "pair": 2}
+TILES = {"auto": 0, "single": 1, "pair": 2, "small": 3}
 
 
 def moe_set_gemm_tiles(mode="auto"):
-    """Process-wide tile shape of the expert GEMMs: 'auto', 'single' (M = 128 per CTA) or
-    'pair' (M = 256 per 2-CTA cluster)."""
+    """Process-wide tile shape of the expert GEMMs: 'auto', 'single' (128-row tiles, one
+    CTA), 'pair' (256-row tiles, 2-CTA cluster) or 'small' (32-row tiles, one CTA)."""
     _check(_set_tiles(TILES[mode] if isinstance(mode, str) else mode), "moe_set_gemm_tiles")
 
 

@@ -134,7 +134,7 @@ const char* moe_status_string(int status) {
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
 moe_status moe_set_gemm_tiles(int mode) {
-  if (mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 3) return MOE_ERR_INVALID_ARG;
   g_tile_mode.store(mode);
   return MOE_OK;
 }

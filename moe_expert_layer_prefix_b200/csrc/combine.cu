@@ -1,4 +1,4 @@
-// Combine kernel: one warp per token (combine.cuh holds the per-token gather-sum and its
+// Combine kernel: one warp per (token, column chunk) (combine.cuh holds the gather-sum and its
 // source).
 #include "combine.cuh"
 #include "common.cuh"
@@ -7,14 +7,19 @@
 namespace moe {
 namespace {
 
-template <bool kF32>
+// One warp per (token, column chunk); nc chunks per token (1: the whole row).
+template <bool kF32, int kV>
 __global__ void __launch_bounds__(256) combine_kernel(const void* __restrict__ y,
                                                       const int32_t* __restrict__ slot_of,
                                                       const float* __restrict__ topk_w, int T,
-                                                      int k, int H, void* __restrict__ out) {
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (t >= T) return;
-  combine_token<kF32>(y, slot_of, topk_w, t, k, H, out, threadIdx.x & 31);
+                                                      int k, int H, void* __restrict__ out,
+                                                      int nc) {
+  const long item = static_cast<long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (item >= static_cast<long>(T) * nc) return;
+  const int t = static_cast<int>(item / nc), c = static_cast<int>(item % nc);
+  const int width = nc == 1 ? H / 8 : 32 * kV;
+  combine_token<kF32, kV>(y, slot_of, topk_w, t, k, H, out, threadIdx.x & 31, c * width,
+                          (c + 1) * width);
 }
 
 // Mixed formats (BF16 y into fp32 out or the reverse) take this simple path.
@@ -48,12 +53,20 @@ cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, con
                            int T, int k, int H, void* out, int out_f32, cudaStream_t s) {
   const int warps = 8;
   count_launch();
-  const dim3 grid((T + warps - 1) / warps), block(32 * warps);
-  if (y_f32 && out_f32)
-    combine_kernel<true><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out);
-  else if (!y_f32 && !out_f32)
-    combine_kernel<false><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out);
-  else
+  // whole rows per warp once there are enough tokens to fill the GPU; column chunks below
+  const bool rows = T >= 4096;
+  const int nc = rows ? 1 : combine_chunks<4>(H);
+  const long items = static_cast<long>(T) * nc;
+  const dim3 block(32 * warps);
+  const dim3 grid(y_f32 == out_f32 ? static_cast<unsigned>((items + warps - 1) / warps)
+                                   : static_cast<unsigned>((T + warps - 1) / warps));
+  if (y_f32 && out_f32) {
+    if (rows) combine_kernel<true, 1><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, 1);
+    else combine_kernel<true, 4><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
+  } else if (!y_f32 && !out_f32) {
+    if (rows) combine_kernel<false, 1><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, 1);
+    else combine_kernel<false, 4><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
+  } else
     combine_mixed_kernel<<<grid, block, 0, s>>>(y, y_f32, slot_of, topk_w, T, k, H, out, out_f32);
   return cudaGetLastError();
 }

@@ -3,8 +3,9 @@
 // The last step of the pages' pipeline puts the expert outputs back together (jiqizhixin,
 // "DeepSeek悄悄更新：Mega MoE、FP4 Indexer来了", section "Mega MoE 是什么？", pipeline
 // paragraph; youleyou, "DeepSeek 模型更新解读 Tile Kernels 与 DeepEP V2 新特性", Tile Kernels
-// feature list, routing item: fused reduce).  One warp per token gathers its k rows and sums
-// them in rank order j in fp32, so the result is deterministic and needs no atomics.
+// feature list, routing item: fused reduce).  A warp takes a chunk of one token's columns,
+// gathers them from the token's k rows and sums in rank order j in fp32, so the result is
+// deterministic and needs no atomics.
 // Shared by the combine kernel and the persistent forward kernel.
 // HBM-bound: reads k rows of y per token, writes one output row, 16-byte accesses.
 #pragma once
@@ -13,16 +14,25 @@
 
 namespace moe {
 
-// One warp computes out[t, :] (all 32 lanes call it together).  y and out are BF16, or fp32
-// for the fp32 layer.  Each lane owns 8 consecutive columns per pass and a warp iteration
-// covers kV passes; the k source rows are read as groups of kJ x kV independent 16-byte
-// loads issued back to back (raw words, converted only afterwards), so a warp keeps many
-// loads in flight even when only a few warps per SM run it.
+// Columns of a token are handed out in chunks of 32 * kV vectors of 8 columns (one warp
+// iteration), so that few tokens still spread over many warps.
+template <int kV>
+__host__ __device__ constexpr int combine_chunks(int H) {
+  return (H / 8 + 32 * kV - 1) / (32 * kV);
+}
+
+// One warp computes out[t, 8*v_begin : 8*v_end] (all 32 lanes call it together; v_begin is a
+// multiple of 32 * kV).  y and out are BF16, or fp32 for the fp32 layer.  Each lane owns 8
+// consecutive columns per pass and a warp iteration covers kV passes; the k source rows are
+// read as groups of kJ x kV independent 16-byte loads issued back to back (raw words,
+// converted only afterwards), so a warp keeps many loads in flight even when only a few
+// warps per SM run it.
 template <bool kF32, int kV = 1>
 __device__ __forceinline__ void combine_token(const void* __restrict__ y,
                                               const int32_t* __restrict__ slot_of,
                                               const float* __restrict__ topk_w, int t, int k,
-                                              int H, void* __restrict__ out, int lane) {
+                                              int H, void* __restrict__ out, int lane,
+                                              int v_begin, int v_end) {
   constexpr int kJ = 8;
   constexpr int kWords = kF32 ? 2 : 1;  // 16-byte words per 8 columns
   int my_slot = 0;
@@ -31,12 +41,12 @@ __device__ __forceinline__ void combine_token(const void* __restrict__ y,
     my_slot = __ldcg(slot_of + static_cast<size_t>(t) * k + lane);
     my_w = __ldcg(topk_w + static_cast<size_t>(t) * k + lane);
   }
-  const int nvec = H / 8;
+  const int nvec = v_end < H / 8 ? v_end : H / 8;
   const uint4* y4 = static_cast<const uint4*>(y);
   const size_t row_words = static_cast<size_t>(H) / 8 * kWords;
   // The trip counts are the same for every lane (the shuffles need the full warp); lanes
   // past the row's end read column 0 and drop the result.
-  for (int v0 = 0; v0 < nvec; v0 += 32 * kV) {
+  for (int v0 = v_begin; v0 < nvec; v0 += 32 * kV) {
     size_t col[kV];
 #pragma unroll
     for (int p = 0; p < kV; ++p) {

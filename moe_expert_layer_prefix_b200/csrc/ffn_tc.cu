@@ -24,9 +24,10 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D K-major tensor map: rows x K, box {128-byte K slice, 128 rows}, 128-byte swizzle.
+// 2-D K-major tensor map: rows x K, box {128-byte K slice, box_rows rows}, 128-byte swizzle.
 // fmt: 0 = BF16, 1 = 8-bit, 2 = E2M1 (expanded to one byte per element in shared memory).
-bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int fmt) {
+bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int fmt,
+                     uint32_t box_rows) {
   EncodeTiledFn fn = encode_fn();
   if (fn == nullptr) return false;
   CUtensorMapDataType dt;
@@ -47,7 +48,7 @@ bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K
   }
   const cuuint64_t dims[2] = {K, rows};
   const cuuint64_t strides[1] = {row_bytes};
-  const cuuint32_t box[2] = {box_k, 128};
+  const cuuint32_t box[2] = {box_k, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -59,21 +60,21 @@ namespace {
 
 using namespace gemm;
 
-template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3>
+template <int kCta, int kTm, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const TcParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const Smem sm = carve<kCta>(smem_raw);
-  gemm_init<kCta, kBlockScaled>(sm, &tmA, 1);
+  const Smem sm = carve<kCta, kTm>(smem_raw);
+  gemm_init<kCta, kBlockScaled, kTm>(sm, &tmA, 1);
   if (threadIdx.x == 0) tma_prefetch_desc(&tmB);
-  gemm_prefix<kCta>(sm, p.offsets, p.E, p.n_tiles);
+  gemm_prefix<kCta, kTm>(sm, p.offsets, p.E, p.n_tiles);
   tc_fence_before();
   __syncthreads();
   if constexpr (kCta == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   Pipe pipe;
-  gemm_phase<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3>(&tmA, &tmB, p, sm, pipe);
+  gemm_phase<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm>(&tmA, &tmB, p, sm, pipe);
   tc_fence_before();
   __syncthreads();
   // in a pair, neither CTA leaves while the other may still touch its shared memory
@@ -85,26 +86,14 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
-// Tile shape: pairs (M = 256) once the average expert holds at least 128 rows; single
-// CTAs (M = 128) for decode-sized batches, where a 256-row tile would be mostly padding.
-// Block-scaled pairs are correct but slower than single CTAs today: every k-step of the
-// peer CTA signals its scale factors to the leader with a cluster-scope release, which
-// throttles the pipeline, so automatic selection keeps them on single CTAs.
-inline bool use_pair(const FfnArgs& a) {
-  const int mode = gemm_tile_mode();
-  if (mode == 1) return false;
-  if (mode == 2) return num_sms() >= 2;
-  return a.act == MOE_BF16 && a.S >= 128 * a.E && num_sms() >= 2;
-}
-
-template <int kCta, bool kBS, int kBFmt, bool kSw, bool kE4>
+template <int kCta, int kTm, bool kBS, int kBFmt, bool kSw, bool kE4>
 cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   const int K = linear1 ? a.H : a.I;
   const int w_rows = linear1 ? 2 * a.I : a.H;
   CUtensorMap tmA, tmB;
   const int afmt = a.act == MOE_BF16 ? 0 : 1;
   const int bfmt = a.wt == MOE_BF16 ? 0 : (a.wt == MOE_E4M3 ? 1 : 2);
-  if (!make_kmajor_map(&tmA, a.a, static_cast<uint64_t>(a.S), static_cast<uint64_t>(K), afmt))
+  if (!make_kmajor_map(&tmA, a.a, static_cast<uint64_t>(a.S), static_cast<uint64_t>(K), afmt, kTm))
     return cudaErrorInvalidValue;
   if (!make_kmajor_map(&tmB, a.w, static_cast<uint64_t>(a.E) * w_rows, static_cast<uint64_t>(K), bfmt))
     return cudaErrorInvalidValue;
@@ -122,8 +111,8 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   p.out = a.out;
   p.out_scales = a.out_scales;
   p.err = a.err;
-  auto kern = grouped_gemm_tc<kCta, kBS, kBFmt, kSw, kE4>;
-  const size_t smem = Cfg<kCta>::kSmem;
+  auto kern = grouped_gemm_tc<kCta, kTm, kBS, kBFmt, kSw, kE4>;
+  const size_t smem = Cfg<kCta, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -145,11 +134,32 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
 
 template <bool kBS, int kBFmt, bool kSw, bool kE4>
 cudaError_t launch_tc_any(const FfnArgs& a, bool linear1, cudaStream_t s) {
-  return use_pair(a) ? launch_tc<2, kBS, kBFmt, kSw, kE4>(a, linear1, s)
-                     : launch_tc<1, kBS, kBFmt, kSw, kE4>(a, linear1, s);
+  switch (gemm_tile_shape(a.act, a.S, a.E, true)) {
+    case 2: return launch_tc<2, kBM, kBS, kBFmt, kSw, kE4>(a, linear1, s);
+    case 3: return launch_tc<1, 32, kBS, kBFmt, kSw, kE4>(a, linear1, s);
+    default: return launch_tc<1, kBM, kBS, kBFmt, kSw, kE4>(a, linear1, s);
+  }
 }
 
 }  // namespace
+
+// Tile shape.  Pairs (M = 256) once the average expert holds at least 128 rows, for BF16:
+// block-scaled pairs are correct but slower than single CTAs (the per-SM k-step rate is the
+// same and the 256-row tiles carry more padding).  Small tiles (32-row m-blocks) when the
+// average expert holds at most 16 rows, as in decode: the weights stream from HBM once per
+// m-block either way, and the smaller A box leaves room for a fifth pipeline stage.
+// Single CTAs (M = 128) otherwise.
+int gemm_tile_shape(int act, int S, int E, bool allow_pair) {
+  int mode = gemm_tile_mode();
+  if (mode == 2 && !allow_pair) mode = 1;
+  if (mode == 1) return 1;
+  if (mode == 2) return num_sms() >= 2 ? 2 : 1;
+  if (mode == 3) return 3;
+  if (static_cast<int64_t>(S) <= 16LL * E) return 3;
+  if (allow_pair && act == MOE_BF16 && static_cast<int64_t>(S) >= 128LL * E && num_sms() >= 2)
+    return 2;
+  return 1;
+}
 
 cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s) {
   if (a.E > kMaxE) return cudaErrorNotSupported;

@@ -52,14 +52,14 @@ struct FwdParams {
   TcParams l1, l2;
 };
 
-template <bool kBS, int kBFmt, bool kE4>
+template <bool kBS, int kBFmt, bool kE4, int kTm>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW2,
                    const FwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const Smem sm = carve<1>(smem_raw);
-  gemm_init<1, kBS>(sm, &tmX, 1);
+  const Smem sm = carve<1, kTm>(smem_raw);
+  gemm_init<1, kBS, kTm>(sm, &tmX, 1);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmH);
@@ -72,11 +72,12 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nwarps = kThreads / 32;
   const int gw = blockIdx.x * nwarps + warp, GW = gridDim.x * nwarps;
-  // dispatch scratch inside the (idle) GEMM ring: per-warp chunk masks in the A stages,
-  // slot tables, scan partials and offsets in the B stages
-  uint32_t* mask = reinterpret_cast<uint32_t*>(sm.sA) + warp * p.E;
-  int32_t(*part)[33] = reinterpret_cast<int32_t(*)[33]>(sm.sB + nwarps * kChunkTokens * 32 * 4);
-  int32_t* soffs = reinterpret_cast<int32_t*>(sm.sB + nwarps * kChunkTokens * 32 * 4 + 32 * 33 * 4);
+  // dispatch scratch inside the (idle) GEMM ring, which is at least 180 KB: per-warp chunk
+  // masks (8 x E words, at most 32 KB), then scan partials, offsets and warp sums
+  uint8_t* scratch = sm.sA;
+  uint32_t* mask = reinterpret_cast<uint32_t*>(scratch) + warp * p.E;
+  int32_t(*part)[33] = reinterpret_cast<int32_t(*)[33]>(scratch + nwarps * kMaxE * 4);
+  int32_t* soffs = reinterpret_cast<int32_t*>(scratch + nwarps * kMaxE * 4 + 32 * 33 * 4);
   int32_t* wsum = soffs + 1028;
 
   // 1. route: one warp per token
@@ -118,25 +119,34 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
 
   // 7. linear-1 + SwiGLU + requantisation
   Pipe pipe;
-  gemm_prefix<1>(sm, p.offsets, p.E, p.l1.n_tiles);
+  gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l1.n_tiles);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  gemm_phase<1, kBS, kBFmt, true, kE4>(&tmX, &tmW1, p.l1, sm, pipe);
+  gemm_phase<1, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
   fence_proxy_async_global();  // h is read by TMA next
   grid_sync(p.bar, p.err);
 
   // 8. linear-2
-  gemm_prefix<1>(sm, p.offsets, p.E, p.l2.n_tiles);
+  gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l2.n_tiles);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  gemm_phase<1, kBS, kBFmt, false, false>(&tmH, &tmW2, p.l2, sm, pipe);
+  gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
   grid_sync(p.bar, p.err);
 
-  // 9. combine: one warp per token
-  for (int t = gw; t < p.T; t += GW)
-    combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane);
+  // 9. combine: one warp per token, or per (token, column chunk) when there are too few
+  //    tokens to keep every warp busy
+  {
+    const int nc = p.T >= 2 * GW ? 1 : combine_chunks<4>(p.H);
+    const int width = nc == 1 ? p.H / 8 : 128;
+    const long items = static_cast<long>(p.T) * nc;
+    for (long it = gw; it < items; it += GW) {
+      const int t = static_cast<int>(it / nc), c = static_cast<int>(it % nc);
+      combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
+                              (c + 1) * width);
+    }
+  }
 
   tc_fence_before();
   __syncthreads();
@@ -144,15 +154,15 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   gemm_fini<1>(sm);
 }
 
-template <bool kBS, int kBFmt, bool kE4>
+template <bool kBS, int kBFmt, bool kE4, int kTm>
 cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   const int S = a.T * a.k;
   const int afmt = a.act == MOE_BF16 ? 0 : 1;
   const int bfmt = a.wt == MOE_BF16 ? 0 : (a.wt == MOE_E4M3 ? 1 : 2);
   CUtensorMap tmX, tmW1, tmH, tmW2;
-  if (!make_kmajor_map(&tmX, a.x_perm, S, a.H, afmt) ||
+  if (!make_kmajor_map(&tmX, a.x_perm, S, a.H, afmt, kTm) ||
       !make_kmajor_map(&tmW1, a.w1, static_cast<uint64_t>(a.E) * 2 * a.I, a.H, bfmt) ||
-      !make_kmajor_map(&tmH, a.h, S, a.I, afmt) ||
+      !make_kmajor_map(&tmH, a.h, S, a.I, afmt, kTm) ||
       !make_kmajor_map(&tmW2, a.w2, static_cast<uint64_t>(a.E) * a.H, a.I, bfmt))
     return cudaErrorInvalidValue;
   FwdParams p;
@@ -206,8 +216,8 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   p.l1 = l1;
   p.l2 = l2;
 
-  auto kern = moe_forward_kernel<kBS, kBFmt, kE4>;
-  const size_t smem = Cfg<1>::kSmem;
+  auto kern = moe_forward_kernel<kBS, kBFmt, kE4, kTm>;
+  const size_t smem = Cfg<1, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;
@@ -232,9 +242,13 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s) {
   // the dispatch phases keep per-warp masks (8 x E words) in the 64 KB of A stages
   if (a.E > 1024) return cudaErrorNotSupported;
-  if (a.act == MOE_BF16 && a.wt == MOE_BF16) return launch<false, 0, false>(a, s);
-  if (a.act == MOE_E4M3 && a.wt == MOE_E4M3) return launch<true, 0, true>(a, s);
-  if (a.act == MOE_E4M3 && a.wt == MOE_E2M1) return launch<true, 5, true>(a, s);
+  const bool small = gemm_tile_shape(a.act, a.T * a.k, a.E, false) == 3;
+  if (a.act == MOE_BF16 && a.wt == MOE_BF16)
+    return small ? launch<false, 0, false, 32>(a, s) : launch<false, 0, false, kBM>(a, s);
+  if (a.act == MOE_E4M3 && a.wt == MOE_E4M3)
+    return small ? launch<true, 0, true, 32>(a, s) : launch<true, 0, true, kBM>(a, s);
+  if (a.act == MOE_E4M3 && a.wt == MOE_E2M1)
+    return small ? launch<true, 5, true, 32>(a, s) : launch<true, 5, true, kBM>(a, s);
   return cudaErrorNotSupported;
 }
 

@@ -54,7 +54,6 @@ namespace gemm {
 constexpr int kBM = 128;           // accumulator rows per CTA (TMEM lanes)
 constexpr int kBN = 256;           // accumulator columns (MMA N)
 constexpr int kRowBytes = 128;     // K bytes per tile row per stage (one swizzle atom)
-constexpr int kATileBytes = kBM * kRowBytes;  // 16 KB
 constexpr int kSfaBytes = 512;     // 128 rows x 4 UE8M0
 constexpr int kSfbBytes = 1024;    // 256 rows x 4 UE8M0
 constexpr int kTmemCols = 512;
@@ -100,12 +99,18 @@ struct SharedState {
   int offs[kMaxE + 1];
 };
 
-template <int kCta>
+// Tile shapes: kCta CTAs per tile, kTm rows of the tile per CTA.  (1, 128) single,
+// (2, 128) pair, (1, 32) small: 32-row m-blocks for decode-sized batches, whose A box is a
+// quarter of the single one, which buys a fifth stage.  The MMA keeps M = 128: rows past
+// kTm read whatever the neighbouring stage holds and their outputs are never stored.
+template <int kCta, int kTm = kBM>
 struct Cfg {
-  static constexpr int kStages = kCta == 2 ? 6 : 4;
+  static_assert(kTm == kBM || (kCta == 1 && kTm == 32), "unsupported tile shape");
+  static constexpr int kStages = kCta == 2 ? 6 : (kTm == kBM ? 4 : 5);
+  static constexpr int kATileBytes = kTm * kRowBytes;     // 16 KB (4 KB small)
   static constexpr int kBRows = kBN / kCta;               // B rows this CTA loads per k-step
   static constexpr int kBTileBytes = kBRows * kRowBytes;  // 32 KB single, 16 KB pair
-  static constexpr int kTileM = kBM * kCta;               // rows of one tile
+  static constexpr int kTileM = kTm * kCta;               // rows of one tile
   static constexpr size_t kSmem = 1024 + kStages * (kATileBytes + kBTileBytes) +
                                   kSfSlots * (kSfaBytes + kSfbBytes) + sizeof(SharedState);
   static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -155,13 +160,13 @@ struct Smem {
   SharedState* ss;
 };
 
-template <int kCta>
+template <int kCta, int kTm = kBM>
 __device__ __forceinline__ Smem carve(uint8_t* smem_raw) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kCta, kTm>;
   Smem m;
   m.sA = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                     ~static_cast<uintptr_t>(1023));
-  m.sB = m.sA + C::kStages * kATileBytes;
+  m.sB = m.sA + C::kStages * C::kATileBytes;
   m.sSF = m.sB + C::kStages * C::kBTileBytes;             // per slot: SFA 512 B, SFB 1024 B
   m.ss = reinterpret_cast<SharedState*>(m.sSF + kSfSlots * (kSfaBytes + kSfbBytes));
   return m;
@@ -169,12 +174,12 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw) {
 
 // Barriers and TMEM; warps 0 and 1.  The caller synchronises the CTA (and the cluster)
 // before any role starts.
-template <int kCta, bool kBlockScaled>
+template <int kCta, bool kBlockScaled, int kTm = kBM>
 __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tmaps, int ntmaps) {
   SharedState& ss = *sm.ss;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == 0 && lane == 0) {
-    for (int s = 0; s < Cfg<kCta>::kStages; ++s) {
+    for (int s = 0; s < Cfg<kCta, kTm>::kStages; ++s) {
       mbar_init(&ss.full[s], 1);
       mbar_init(&ss.empty[s], 1);
     }
@@ -202,10 +207,10 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
 }
 
 // Tile list of one GEMM from the expert offsets (warp 3; the caller synchronises after).
-template <int kCta>
+template <int kCta, int kTm = kBM>
 __device__ __forceinline__ void gemm_prefix(const Smem& sm, const int32_t* offsets, int E,
                                             int n_tiles) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kCta, kTm>;
   SharedState& ss = *sm.ss;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp != 3) return;
@@ -245,10 +250,10 @@ __device__ __forceinline__ void gemm_fini(const Smem& sm) {
 // kCta: 1 (single) or 2 (pair).  kBlockScaled: false -> BF16 kind::f16; true ->
 // kind::mxf8f6f4 with A = E4M3 and B = E4M3 (kBFmt 0) or E2M1 (kBFmt 5).  kSwiGLU: linear-1
 // epilogue, else linear-2.  kOutE4M3: linear-1 stores h as E4M3 + 1x128 scales (else BF16).
-template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3>
+template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm = kBM>
 __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
                                            const TcParams& p, const Smem& sm, Pipe& pipe) {
-  using C = Cfg<kCta>;
+  using C = Cfg<kCta, kTm>;
   constexpr bool kPair = kCta == 2;
   constexpr int kStages = C::kStages;
   const CUtensorMap& tmA = *tmA_;
@@ -271,12 +276,12 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       constexpr uint32_t kBBytes = kBFmt == 5 ? C::kBTileBytes / 2 : C::kBTileBytes;
-      constexpr uint32_t kCtaBytes = kATileBytes + kBBytes;
+      constexpr uint32_t kCtaBytes = C::kATileBytes + kBBytes;
       uint32_t it = pipe.prod_it;
       const uint32_t it0 = it;
       for (int t = cid; t < total && !*abort; t += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
-        const int arow = tile.m0 + static_cast<int>(rank) * kBM;
+        const int arow = tile.m0 + static_cast<int>(rank) * kTm;
         // B rows of this CTA: linear-1 gate rows [nb*128, +128) then up rows [I + nb*128, +128);
         // linear-2 rows [nb*256, +256); a pair splits them between its two CTAs
         const int ebase = tile.e * p.w_rows;
@@ -291,11 +296,11 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           if constexpr (kPair) {
             if (rank == 0) mbar_arrive_expect_tx(&ss.full[stage], 2 * kCtaBytes);
             const uint32_t bar = mapa_shared(smem_u32(&ss.full[stage]), 0);
-            tma_load_2d_pair(sA + stage * kATileBytes, &tmA, bar, kx, arow);
+            tma_load_2d_pair(sA + stage * C::kATileBytes, &tmA, bar, kx, arow);
             tma_load_2d_pair(sB + stage * C::kBTileBytes, &tmB, bar, kx, brow);
           } else {
             mbar_arrive_expect_tx(&ss.full[stage], kCtaBytes);
-            tma_load_2d(sA + stage * kATileBytes, &tmA, &ss.full[stage], kx, arow);
+            tma_load_2d(sA + stage * C::kATileBytes, &tmA, &ss.full[stage], kx, arow);
             tma_load_2d(sB + stage * C::kBTileBytes, &tmB, &ss.full[stage], kx, g0);
             tma_load_2d(sB + stage * C::kBTileBytes + C::kBTileBytes / 2, &tmB, &ss.full[stage], kx,
                         g1);
@@ -357,7 +362,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             }
           }
           tc_fence_after();
-          const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * kATileBytes));
+          const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * C::kATileBytes));
           const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
           if (grp_start) ++grp;
           // A scales (and E4M3 B scales) are per 128 of K, so one byte per k-step: a group of
@@ -590,8 +595,8 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           mbar_wait<kPair>(&ss.acc_full, acc_phase, p.err, SITE_GEMM_ACC_FULL, abort);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
-      const int row = tile.m0 + static_cast<int>(rank) * kBM + q * 32 + lane;
-      const bool valid = row < tile.m_end;
+      const int row = tile.m0 + static_cast<int>(rank) * kTm + q * 32 + lane;
+      const bool valid = q * 32 + lane < kTm && row < tile.m_end;
       if constexpr (kSwiGLU) {
         if constexpr (kOutE4M3) {
           float h[128];

@@ -52,7 +52,8 @@ cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s);
 
 // 2-D K-major tensor map: rows x K, box {128-byte K slice, 128 rows}, 128-byte swizzle.
 // fmt: 0 = BF16, 1 = 8-bit, 2 = E2M1 (expanded to one byte per element in shared memory).
-bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int fmt);
+bool make_kmajor_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t K, int fmt,
+                     uint32_t box_rows = 128);
 
 // The whole layer in one persistent cooperative launch (tensor-core formats only);
 // returns cudaErrorNotSupported when the layer cannot run that way.
@@ -86,7 +87,10 @@ struct ForwardArgs {
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s);
 
 int* device_error_word();   // device address of the calling device's error word
-int gemm_tile_mode();       // 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles
+int gemm_tile_mode();
+// Tile shape for a grouped GEMM over S rows and E experts: 1 single, 2 pair, 3 small (32-row
+// m-blocks).  allow_pair = false where only single-CTA shapes exist (the persistent kernel).
+int gemm_tile_shape(int act, int S, int E, bool allow_pair);       // 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles
 int num_sms();
 
 }  // namespace moe

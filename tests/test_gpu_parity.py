@@ -31,14 +31,28 @@ SMALL = {
     "mixtral_bf16_h384_pair": synth.WORKLOADS["mixtral_bf16"].scaled(T=400, H=384, E=3, I=256),
     "skewed_fp8_fp4_pair": synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=512, H=512, E=32, k=8,
                                                                     I=256),
+    # 32-row tiles forced on shapes that would not pick them (several m-blocks per expert)
+    "v3_fp8_small": synth.WORKLOADS["v3_fp8"].scaled(T=300, H=1024, E=16, k=4, I=512),
+    "skewed_fp8_fp4_small": synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=260, H=512, E=128,
+                                                                     I=256),
+    "mixtral_bf16_h384_small": synth.WORKLOADS["mixtral_bf16"].scaled(T=77, H=384, E=5, I=256),
 }
 
 
 @pytest.fixture(autouse=True)
-def _clear_device_error():
-    """Each test starts with a clear device error word (and asserts on its own errors)."""
+def _clear_device_error(request):
+    """Each test starts with a clear device error word (and asserts on its own errors);
+    configurations named *_small run with 32-row tiles forced."""
     M.moe_get_device_error()
-    yield
+    name = getattr(request.node, "callspec", None)
+    small = name is not None and str(name.params.get("name", "")).endswith("_small")
+    if small:
+        M.moe_set_gemm_tiles("small")
+    try:
+        yield
+    finally:
+        if small:
+            M.moe_set_gemm_tiles("auto")
 
 
 def _inputs(wl):
@@ -221,14 +235,16 @@ def test_forward_end_to_end(name):
 
 
 @pytest.mark.parametrize("name", ["v3_fp8", "skewed_fp8_fp4", "mixtral_bf16",
-                                  "v3_fp8_pair", "skewed_fp8_fp4_pair"])
+                                  "v3_fp8_pair", "skewed_fp8_fp4_pair", "decode_fp8_fp4",
+                                  "v3_fp8_small"])
 def test_forward_equals_unfused_chain(name):
     """moe_forward (one persistent launch) produces exactly the bytes of the chain of entry
-    points (same device code, same tile order; single-CTA tiles for both)."""
+    points (same device code, same tile order; the same single-CTA tile shape for both)."""
     wl = SMALL[name]
     d = _inputs(wl)
     W = weights_of(wl, d)
-    M.moe_set_gemm_tiles("single")
+    M.moe_set_gemm_tiles("small" if name.endswith("_small") or name.startswith("decode")
+                         else "single")
     try:
         idx1 = torch.empty((wl.T, wl.k), dtype=torch.int32, device=DEV)
         out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
@@ -244,6 +260,33 @@ def test_forward_equals_unfused_chain(name):
         M.moe_set_gemm_tiles("auto")
     assert torch.equal(idx1, idx)
     assert torch.equal(out, out2)
+
+
+@pytest.mark.parametrize("name", ["v3_fp8", "skewed_fp8_fp4", "mixtral_bf16_h384"])
+def test_small_tiles_equal_single(name):
+    """32-row and 128-row tiles run the same M = 128 MMAs over the same K order on each
+    row, so the expert GEMMs give the same bits either way."""
+    wl = SMALL[name]
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    idx, _ = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+    r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+    res = []
+    try:
+        for mode in ("single", "small"):
+            M.moe_set_gemm_tiles(mode)
+            h, hs = M.moe_expert_linear1(r["x_perm"], r["expert_offsets"], W,
+                                         x_perm_scales=r["x_perm_scales"])
+            y = M.moe_expert_linear2(h, r["expert_offsets"], W, h_scales=hs)
+            torch.cuda.synchronize()
+            assert M.moe_get_device_error()[0] == 0
+            res.append((h, hs, y))
+    finally:
+        M.moe_set_gemm_tiles("auto")
+    (h1, hs1, y1), (h2, hs2, y2) = res
+    assert torch.equal(h1, h2)
+    assert hs1 is None or torch.equal(hs1, hs2)
+    assert torch.equal(y1, y2)
 
 
 def test_forward_deterministic():
