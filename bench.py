@@ -33,6 +33,13 @@ import synth  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
+# DRAM traffic of a kernel as a multiple of its algorithmic bytes, from an ncu capture of a
+# smaller case with the same rows per expert (dram__bytes_read.sum + dram__bytes_write.sum
+# of one launch).  Used for the roofline's "traffic".
+TRAFFIC_RATIO = {
+    ("v3_fp8", "linear1"): (1.154, "the V3-shaped layer at T=1024, E=32"),
+}
+
 
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -328,7 +335,15 @@ def run_native(args, ws, rank, local):
                 "peak": pk["hbm_gbs"], "unit": "GB/s", "peak_note": f"{pk_kind} copy bandwidth"}
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["kernel"] = dom
-    roof["traffic"] = args.traffic
+    if args.traffic is not None:
+        roof["traffic"] = args.traffic
+    elif (wl.name, dom) in TRAFFIC_RATIO:
+        ratio, src = TRAFFIC_RATIO[(wl.name, dom)]
+        roof["traffic"] = ratio * alg[dom]["bytes"]
+        roof["traffic_note"] = (f"DRAM read+write bytes per launch = {ratio} x algorithmic, "
+                                f"the ratio ncu measured on {src}")
+    else:
+        roof["traffic"] = None
     roof["algorithmic_per_launch"] = {"bytes": alg[dom]["bytes"], "flops": alg[dom]["flops"]}
 
     res = {
