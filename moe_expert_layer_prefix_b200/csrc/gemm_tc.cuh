@@ -9,8 +9,9 @@
 // Both GEMMs have the form  D[m, n] = sum_k A[m, k] * B[n, k]  per expert, A = the expert's
 // rows of x_perm (or h), B = the expert's K-major weight matrix.  Persistent CTAs (one per
 // SM) walk a static list of output tiles (expert, m-block, n-block) of N = 256 columns.
-// Two tile shapes:
+// Tile shapes (Cfg below):
 //   single  one CTA, M = 128: A 128 x 128 B and B 256 x 128 B per k-step, 4 stages
+//   small   one CTA, 32-row m-blocks: a 32-row A box, 5 stages
 //   pair    a 2-CTA cluster, M = 256 (tcgen05 cta_group::2): each CTA loads its own 128 A
 //           rows and half of the B rows (128 x 128 B) per k-step, 6 stages; the leader CTA
 //           issues the MMAs, which read both CTAs' shared memory and write both CTAs' TMEM,
@@ -22,10 +23,10 @@
 //   warp 1      MMA issuer (one thread, leader CTA): tcgen05.mma 128|256 x 256 x {16|32}
 //               into a TMEM fp32 accumulator (256 columns); tcgen05.commit frees ring stages
 //               (in both CTAs of a pair)
-//   warp 2      scale loader (block-scaled kinds): prefetches the raw scale words of each
-//               k-step into a small shared-memory ring
-//   warp 3      scale converter: UE8M0 words in the layout tcgen05.cp reads, then signals the
-//               (leader's) stage barrier; before the first phase it also builds the tile list
+//   warp 2      scale loader (block-scaled kinds): copies the raw scale words of each k-step
+//               into a 16-slot shared-memory ring with asynchronous 4-byte copies (cp.async)
+//   warp 3      scale converter: UE8M0 bytes in the layout tcgen05.cp reads, then signals the
+//               (leader's) slot barriers; before each GEMM phase it also builds the tile list
 //   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp i reads TMEM lanes 32i..32i+31,
 //               one output row per thread), SwiGLU + BF16 / E4M3 requantisation (linear-1)
 //               or BF16 conversion (linear-2), 16-byte global stores
