@@ -143,6 +143,72 @@ __device__ __forceinline__ float silu_mul(float g, float u) {
   return __fdividef(g * u, 1.0f + __expf(-g));
 }
 
+// Epilogue stores of linear-2.  Each epilogue thread owns one output row (its TMEM lane), so
+// stores straight from registers write 16 bytes into each of 32 rows per warp instruction:
+// half sectors, which the memory system takes far more slowly than whole ones (linear-2's
+// 512-byte rows of y made the whole GEMM up to 40 % slower).  Instead each pair of lanes
+// swaps halves of kEpiGroup x kEpiGroup blocks of 16-byte chunks with shuffles (one butterfly
+// stage per doubling of kEpiGroup), after which store instruction j of a group writes
+// 16 * kEpiGroup contiguous bytes of the group's row j: whole 32-byte sectors for pairs.
+// (Groups of 4 measured the same, groups of 8 slower: the shuffles share the issue path with
+// the pipeline's barrier traffic.  linear-1's 128-byte h rows keep the direct stores, which
+// measured faster there.)
+constexpr int kEpiGroup = 2;
+
+// w holds the thread's row as 16-byte chunks (chunk c = words 4c..4c+3); block kB is chunks
+// kEpiGroup*kB .. +kEpiGroup-1.  Afterwards thread i of its group holds, in chunk slot
+// kEpiGroup*kB + j, the chunk kEpiGroup*kB + i of the group's row j.
+template <int kB, int kN>
+__device__ __forceinline__ void transpose_block(uint32_t (&w)[kN], int lane) {
+#pragma unroll
+  for (int k = 1; k < kEpiGroup; k <<= 1) {
+    const bool upper = (lane & k) != 0;
+#pragma unroll
+    for (int j = 0; j < kEpiGroup; ++j) {
+      if (j & k) continue;
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint32_t& lo = w[4 * (kEpiGroup * kB + j) + v];
+        uint32_t& hi = w[4 * (kEpiGroup * kB + (j ^ k)) + v];
+        const uint32_t y = __shfl_xor_sync(0xffffffffu, upper ? lo : hi, k);
+        if (upper) lo = y;
+        else hi = y;
+      }
+    }
+  }
+}
+
+template <int kB, int kBlocks, int kN>
+__device__ __forceinline__ void store_blocks(uint32_t (&w)[kN], uint8_t* lane_base, size_t pitch,
+                                             int rows_left, int chunks_left, int lane) {
+  if constexpr (kB < kBlocks) {
+    transpose_block<kB>(w, lane);
+#pragma unroll
+    for (int j = 0; j < kEpiGroup; ++j) {
+      if (j < rows_left && kEpiGroup * kB < chunks_left)
+        *reinterpret_cast<uint4*>(lane_base + j * pitch + 16 * kEpiGroup * kB) =
+            make_uint4(w[4 * (kEpiGroup * kB + j)], w[4 * (kEpiGroup * kB + j) + 1],
+                       w[4 * (kEpiGroup * kB + j) + 2], w[4 * (kEpiGroup * kB + j) + 3]);
+    }
+    store_blocks<kB + 1, kBlocks>(w, lane_base, pitch, rows_left, chunks_left, lane);
+  }
+}
+
+// Stores the warp's 32 rows of kChunks 16-byte chunks.  row0 points at the warp's first row
+// (lane 0's), pitch is the row pitch in bytes, rows_ok the number of leading rows of the warp
+// that exist, chunks_ok the number of leading chunks inside the output (both warp-uniform).
+template <int kChunks>
+__device__ __forceinline__ void store_rows_coalesced(uint32_t (&w)[4 * kChunks], uint8_t* row0,
+                                                     size_t pitch, int rows_ok, int chunks_ok,
+                                                     int lane) {
+  static_assert(kChunks % kEpiGroup == 0, "chunks come in whole blocks");
+  const int g = lane / kEpiGroup, i = lane % kEpiGroup;
+  // this lane writes rows kEpiGroup*g + j and chunks kEpiGroup*b + i
+  uint8_t* lane_base = row0 + static_cast<size_t>(kEpiGroup * g) * pitch + 16 * i;
+  store_blocks<0, kChunks / kEpiGroup>(w, lane_base, pitch, rows_ok - kEpiGroup * g,
+                                       chunks_ok - i, lane);
+}
+
 // Per-thread pipeline counters.  Each role advances only its own; they carry over from one
 // GEMM phase to the next inside a kernel so that the mbarrier phase parities stay in step.
 struct Pipe {
@@ -596,8 +662,11 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           mbar_wait<kPair>(&ss.acc_full, acc_phase, p.err, SITE_GEMM_ACC_FULL, abort);
       if (!__all_sync(0xffffffffu, ready)) break;
       tc_fence_after();
-      const int row = tile.m0 + static_cast<int>(rank) * kTm + q * 32 + lane;
+      const int row0 = tile.m0 + static_cast<int>(rank) * kTm + q * 32;  // the warp's first row
+      const int row = row0 + lane;
       const bool valid = q * 32 + lane < kTm && row < tile.m_end;
+      // rows of this warp that exist (the tile's rows of this CTA, up to the expert's end)
+      const int rows_ok = min(kTm - q * 32, tile.m_end - row0);
       if constexpr (kSwiGLU) {
         if constexpr (kOutE4M3) {
           float h[128];
@@ -696,20 +765,12 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
           else mbar_arrive(&ss.acc_empty);
         }
-        if (valid) {
-          __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) + static_cast<size_t>(row) * p.n_out;
-#pragma unroll
-          for (int c = 0; c < kBN / 32; ++c) {
-            const int col = tile.nb * kBN + 32 * c;
-            if (col < p.n_out) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-#pragma unroll
-              for (int v = 0; v < 4; ++v)
-                dst[v] = make_uint4(w[16 * c + 4 * v], w[16 * c + 4 * v + 1], w[16 * c + 4 * v + 2],
-                                    w[16 * c + 4 * v + 3]);
-            }
-          }
-        }
+        // chunk k of the row = words 4k..4k+3 = columns nb*256 + 8k .. + 8
+        const int chunks_ok = min(kBN / 8, (p.n_out - tile.nb * kBN) / 8);
+        store_rows_coalesced<kBN / 8>(
+            w, reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) +
+                                          static_cast<size_t>(row0) * p.n_out + tile.nb * kBN),
+            static_cast<size_t>(p.n_out) * 2, rows_ok, chunks_ok, lane);
       }
       ++tiles;
     }
