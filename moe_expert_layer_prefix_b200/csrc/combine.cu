@@ -53,20 +53,18 @@ cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, con
                            int T, int k, int H, void* out, int out_f32, cudaStream_t s) {
   const int warps = 8;
   count_launch();
-  // whole rows per warp once there are enough tokens to fill the GPU; column chunks below
-  const bool rows = T >= 4096;
-  const int nc = rows ? 1 : combine_chunks<4>(H);
+  // one warp per 512 columns of a token with two 16-byte loads per lane and source row in
+  // flight per pass: the fastest of the shapes measured on the V3, skewed and decode layers
+  const int nc = combine_chunks<2>(H);
   const long items = static_cast<long>(T) * nc;
   const dim3 block(32 * warps);
   const dim3 grid(y_f32 == out_f32 ? static_cast<unsigned>((items + warps - 1) / warps)
                                    : static_cast<unsigned>((T + warps - 1) / warps));
-  if (y_f32 && out_f32) {
-    if (rows) combine_kernel<true, 1><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, 1);
-    else combine_kernel<true, 4><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
-  } else if (!y_f32 && !out_f32) {
-    if (rows) combine_kernel<false, 1><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, 1);
-    else combine_kernel<false, 4><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
-  } else
+  if (y_f32 && out_f32)
+    combine_kernel<true, 2><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
+  else if (!y_f32 && !out_f32)
+    combine_kernel<false, 2><<<grid, block, 0, s>>>(y, slot_of, topk_w, T, k, H, out, nc);
+  else
     combine_mixed_kernel<<<grid, block, 0, s>>>(y, y_f32, slot_of, topk_w, T, k, H, out, out_f32);
   return cudaGetLastError();
 }

@@ -135,15 +135,20 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
   grid_sync(p.bar, p.err);
 
-  // 9. combine: one warp per token, or per (token, column chunk) when there are too few
-  //    tokens to keep every warp busy
-  {
-    const int nc = p.T >= 2 * GW ? 1 : combine_chunks<4>(p.H);
-    const int width = nc == 1 ? p.H / 8 : 128;
+  // 9. combine.  With only 8 warps per SM here, a warp keeps four 16-byte loads per lane and
+  //    source row in flight and takes a whole token when there are tokens enough for every
+  //    warp; fewer tokens are split into 512-column chunks with two loads in flight (the
+  //    faster of the shapes measured on the V3, skewed and decode layers).
+  if (p.T >= 2 * GW) {
+    for (int t = gw; t < p.T; t += GW)
+      combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
+  } else {
+    const int nc = combine_chunks<2>(p.H);
+    const int width = nc == 1 ? p.H / 8 : 64;
     const long items = static_cast<long>(p.T) * nc;
     for (long it = gw; it < items; it += GW) {
       const int t = static_cast<int>(it / nc), c = static_cast<int>(it % nc);
-      combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
+      combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
                               (c + 1) * width);
     }
   }
