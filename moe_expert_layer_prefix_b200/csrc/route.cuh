@@ -83,35 +83,66 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
     }
   }
 
+  // Selection.  A candidate is packed into one 64-bit word ordered like (key, id): the key
+  // as an order-preserving integer in the high half (-0 taken as +0, so that equal keys give
+  // equal words), the complemented id in the low half (lower id wins a tie).  0 is below
+  // every candidate.  Each lane caches its best two untaken candidates; a round takes the
+  // warp maximum of the lanes' best (5 shuffle steps), the winning lane moves its second
+  // up, and only a lane that wins twice in a row rescans its NPL experts.
+  auto pack = [](float key, int e) -> uint64_t {
+    uint32_t u = __float_as_uint(__fadd_rn(key, 0.0f));
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+    return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~e);
+  };
   uint32_t taken = 0;
+  uint64_t b1 = 0, b2 = 0;  // this lane's best and second-best untaken candidates
+  float v1 = 0.0f, v2 = 0.0f;
+  auto scan = [&]() {
+    b1 = b2 = 0;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && !((taken >> i) & 1u)) {
+        const uint64_t c = pack(key[i], e);
+        if (c > b1) {
+          b2 = b1;
+          v2 = v1;
+          b1 = c;
+          v1 = val[i];
+        } else if (c > b2) {
+          b2 = c;
+          v2 = val[i];
+        }
+      }
+    }
+  };
+  scan();
+  bool second_ok = true;  // b2 is this lane's true second best
   int my_idx = 0;      // lane j keeps the j-th selection
   float my_val = 0.0f;
   float top_val = 0.0f;
   for (int j = 0; j < k; ++j) {
-    float bk = -INFINITY;
-    int bi = 0x7FFFFFFF;
-    float bv = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u) && better(key[i], e, bk, bi)) {
-        bk = key[i];
-        bi = e;
-        bv = val[i];
-      }
-    }
+    uint64_t best = b1;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-      if (better(ok, oi, bk, bi)) {
-        bk = ok;
-        bi = oi;
-        bv = ov;
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+      best = o > best ? o : best;
+    }
+    const int bi = static_cast<int>(~static_cast<uint32_t>(best));
+    const int owner = bi & 31;
+    const float bv = __shfl_sync(0xffffffffu, v1, owner);
+    if (lane == owner) {
+      taken |= 1u << (bi >> 5);
+      if (second_ok) {
+        b1 = b2;
+        v1 = v2;
+        b2 = 0;
+        second_ok = false;
+      } else {
+        scan();
+        second_ok = true;
       }
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (lane == j) {
       my_idx = bi;
       my_val = bv;
