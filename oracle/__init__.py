@@ -39,11 +39,11 @@ from .formats import (e4m3_decode, e4m3_encode, e2m1_decode_packed, ue8m0_decode
                       bf16_bits_to_f64, round_bf16, round_bf16_bits)
 from .fexp import exp_f32, sigmoid_f32
 from .moe import (route, dispatch, dequant_x, dequant_w, quant_e4m3_1x128, expert_ffn,
-                  combine, forward, forward_tokens, ffn_slots, Layer)
+                  combine, forward, forward_tokens, ffn_slots, Layer, quantize_activations)
 
 __all__ = [
     "e4m3_decode", "e4m3_encode", "e2m1_decode_packed", "ue8m0_decode", "bf16_bits_to_f64",
     "round_bf16", "round_bf16_bits", "exp_f32", "sigmoid_f32", "route", "dispatch",
     "dequant_x", "dequant_w", "quant_e4m3_1x128", "expert_ffn", "combine", "forward",
-    "forward_tokens", "ffn_slots", "Layer",
+    "forward_tokens", "ffn_slots", "Layer", "quantize_activations",
 ]

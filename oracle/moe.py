@@ -15,6 +15,9 @@ Steps and the passages they follow:
                 per-block quantisation fused with SwiGLU).
 4. combine   -- jiqizhixin, same section, pipeline paragraph (results are put back
                 together); youleyou, routing item (fused reduce).
+0. (before dispatch, for BF16 input to an E4M3 layer) activation quantisation -- youleyou,
+                feature list, quantisation item (FP8 per-block quantisation); jiqizhixin,
+                FP8 x FP4 paragraph (FP8 activations): quantize_activations.
 
 Tensor formats follow the layer's data contract:
   x      [T, H]   f32 | bf16 bits (uint16) | E4M3 codes (uint8) + x_scales f32 [T, H/128]
@@ -139,14 +142,17 @@ def dequant_w(w, w_scales, wt: str) -> np.ndarray:
 # 3. expert FFN
 # ----------------------------------------------------------------------------------------
 def _pow2_scale_exponent(amax: np.ndarray) -> np.ndarray:
-    """Smallest integer n with amax <= 448 * 2^n (n = 0 where amax == 0)."""
+    """Smallest integer n with amax <= 448 * 2^n (n = 0 where amax == 0), but at least -126:
+    the scale 2^n is stored as a normal fp32 value (and read as its UE8M0 exponent byte), so
+    blocks with amax below 448 * 2^-127 (about 2.6e-36) take 2^-126 and their codes round
+    from amax * 2^126 < 224."""
     a = np.asarray(amax, np.float64)
     safe = np.where(a > 0, a, E4M3_MAX)
     n = np.ceil(np.log2(safe / E4M3_MAX)).astype(np.int64)
     # make the defining inequality exact whatever log2 rounded to
     n = np.where(safe > np.ldexp(E4M3_MAX, n), n + 1, n)
     n = np.where(safe <= np.ldexp(E4M3_MAX, n - 1), n - 1, n)
-    return np.where(a > 0, n, 0)
+    return np.where(a > 0, np.maximum(n, -126), 0)
 
 
 def quant_e4m3_1x128(h32):
@@ -163,6 +169,14 @@ def quant_e4m3_1x128(h32):
     scales = np.ldexp(1.0, ex)
     codes = e4m3_encode(blocks / scales[:, :, None]).reshape(n_rows, C)
     return codes, scales.astype(np.float32)
+
+
+def quantize_activations(x_bf16_bits):
+    """BF16 token rows (uint16 bits [T, H]) -> E4M3 codes [T, H] + fp32 scales [T, H/128],
+    one power-of-two scale per 1x128 block by the same rule as h (quant_e4m3_1x128).  BF16
+    values are exact in fp32, so the result depends on the input bits alone."""
+    x32 = bf16_bits_to_f64(np.asarray(x_bf16_bits, np.uint16)).astype(np.float32)
+    return quant_e4m3_1x128(x32)
 
 
 def _store_h(h: np.ndarray, act: str) -> np.ndarray:
