@@ -113,6 +113,22 @@ moe_status moe_dispatch(const void* x, const float* x_scales, int act, int T, in
                         int32_t* expert_offsets, int32_t* perm_src, int32_t* slot_of, void* ws,
                         size_t ws_bytes, cudaStream_t stream);
 
+/* Dispatch of BF16 rows into an E4M3 layer: moe_dispatch with the activation quantisation
+ * fused into the row copy.  Each 1x128 block of a token row gets the scale 2^n, n the
+ * smallest integer with amax <= 448 * 2^n (an all-zero block gets 2^0; n >= -126), and codes
+ * round to nearest even, saturating — the rule of the h requantisation; the codes are a
+ * function of the input bits alone.
+ * (youleyou, "DeepSeek 模型更新解读 Tile Kernels 与 DeepEP V2 新特性", Tile Kernels feature
+ *  list, quantisation item: FP8 per-block quantisation; jiqizhixin, "DeepSeek悄悄更新：Mega
+ *  MoE、FP4 Indexer来了", FP8 x FP4 paragraph: FP8 activations.)
+ *   x              BF16 [T, H] (16-byte aligned)
+ *   x_perm         E4M3 codes [S, H] out;  x_perm_scales fp32 [S, H/128] out
+ *   other arguments, outputs, workspace and errors as moe_dispatch. */
+moe_status moe_dispatch_quant(const void* x, int T, int H, int E, int k,
+                              const int32_t* topk_idx, void* x_perm, float* x_perm_scales,
+                              int32_t* expert_offsets, int32_t* perm_src, int32_t* slot_of,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* Expert linear-1 + SwiGLU (+ requantisation): for every slot p of expert e,
  *   gate = x_perm[p] . W1[e, 0:I]^T, up = x_perm[p] . W1[e, I:2I]^T (fp32 accumulation),
  *   h[p] = silu(gate) * up stored in format W->act; for E4M3 each 1x128 block of h gets the
@@ -158,7 +174,9 @@ moe_status moe_combine(const void* y, int y_dt, const int32_t* slot_of, const fl
  * it produces the same bytes as the chain moe_route, moe_dispatch, moe_expert_linear1,
  * moe_expert_linear2, moe_combine.  The fp32 layer runs that chain.
  * topk_idx / topk_w / expert_offsets may be NULL; when given, the routing result and the
- * per-expert offsets are written there too. */
+ * per-expert offsets are written there too.
+ * x is in format W->act with x_scales for E4M3; for E4M3 layers x_scales may instead be NULL,
+ * and then x is BF16 [T, H] that the dispatch quantises as moe_dispatch_quant does. */
 moe_status moe_forward(const void* x, const float* x_scales, const float* logits,
                        const float* bias, int score, int renorm, int T, int H, int E, int k,
                        int I, const moe_weights* W, void* out, int32_t* topk_idx,

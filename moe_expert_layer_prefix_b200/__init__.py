@@ -34,7 +34,7 @@ OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5}
 EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
            "moe_get_device_error", "moe_status_string", "moe_launch_count",
-           "moe_dispatch_noalloc", "moe_set_gemm_tiles")
+           "moe_dispatch_noalloc", "moe_set_gemm_tiles", "moe_dispatch_quant")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -61,6 +61,8 @@ _fused_ffn = _sig("moe_fused_ffn", _I, [_P, _P, _P, _I, _I, _I, _I, ctypes.POINT
                                         _P, _P, _Z, _P])
 _dispatch_noalloc = _sig("moe_dispatch_noalloc", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P,
                                                       _P, _P, _P, _P])
+_dispatch_quant = _sig("moe_dispatch_quant", _I, [_P, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
+                                                  _Z, _P])
 _combine = _sig("moe_combine", _I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _P])
 _forward = _sig("moe_forward", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                     ctypes.POINTER(MoeWeights), _P, _P, _P, _P, _P, _Z, _P])
@@ -243,6 +245,8 @@ def moe_combine(y, slot_of, topk_w, out=None, out_dtype=None, stream=None):
 def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=True,
                 x_scales=None, out=None, ws=None, topk_idx=None, topk_w=None,
                 expert_offsets=None, stream=None):
+    """The whole layer.  For an E4M3 layer, x is either E4M3 codes with x_scales, or BF16 with
+    x_scales=None (quantised by the dispatch)."""
     T, H = x.shape
     E = logits.shape[1]
     dev = x.device
@@ -257,6 +261,29 @@ def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=Tru
                     _ptr(topk_w), _ptr(expert_offsets), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return out
+
+
+def moe_dispatch_quant(x, topk_idx, E, ws=None, stream=None):
+    """Dispatch of BF16 rows x [T, H] into an E4M3 layer, quantising on the way (1x128
+    power-of-two scales).  Returns dict(x_perm (E4M3 codes, uint8), x_perm_scales,
+    expert_offsets, perm_src, slot_of)."""
+    T, H = x.shape
+    k = topk_idx.shape[1]
+    S = T * k
+    dev = x.device
+    r = {"x_perm": torch.empty((S, H), dtype=torch.uint8, device=dev),
+         "x_perm_scales": torch.empty((S, H // 128), dtype=torch.float32, device=dev),
+         "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
+         "perm_src": torch.empty(S, dtype=torch.int32, device=dev),
+         "slot_of": torch.empty(S, dtype=torch.int32, device=dev)}
+    need = moe_workspace_size("dispatch", T, H, E, k, 128, "e4m3", "e4m3")
+    if ws is None:
+        ws = workspace(need, dev)
+    _check(_dispatch_quant(_ptr(x), T, H, E, k, _ptr(topk_idx), _ptr(r["x_perm"]),
+                           _ptr(r["x_perm_scales"]), _ptr(r["expert_offsets"]),
+                           _ptr(r["perm_src"]), _ptr(r["slot_of"]), _ptr(ws), ws.numel(),
+                           _stream(stream)), "moe_dispatch_quant")
+    return r
 
 
 def moe_dispatch_noalloc(x, topk_idx, E, act, out, x_scales=None, stream=None):

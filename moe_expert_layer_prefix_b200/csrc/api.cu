@@ -217,6 +217,23 @@ moe_status moe_dispatch(const void* x, const float* x_scales, int act, int T, in
                                      perm_src, slot_of, ws, stream));
 }
 
+moe_status moe_dispatch_quant(const void* x, int T, int H, int E, int k,
+                              const int32_t* topk_idx, void* x_perm, float* x_perm_scales,
+                              int32_t* expert_offsets, int32_t* perm_src, int32_t* slot_of,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+  moe_status st = check_shapes(T, H, E, k);
+  if (st != MOE_OK) return st;
+  if (!x || !topk_idx || !x_perm || !x_perm_scales || !expert_offsets || !perm_src || !slot_of)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(x_perm, 16) || !aligned(x_perm_scales, 4) ||
+      !aligned(topk_idx, 4) || !aligned(expert_offsets, 4) || !aligned(perm_src, 4) ||
+      !aligned(slot_of, 4))
+    return MOE_ERR_MISALIGNED;
+  if (!ws || !aligned(ws, 256) || ws_bytes < dispatch_ws_bytes(T, E)) return MOE_ERR_WORKSPACE;
+  return cuda_status(launch_dispatch(x, nullptr, H, T, H, E, k, topk_idx, x_perm, x_perm_scales,
+                                     expert_offsets, perm_src, slot_of, ws, stream, true));
+}
+
 static moe_status check_ffn(const void* a, const float* a_scales, const int32_t* offsets, int S,
                             int H, int I, int E, const moe_weights* W, const void* out) {
   if (!a || !offsets || !out) return MOE_ERR_INVALID_ARG;
@@ -300,7 +317,7 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
   st = check_weights(W, -1);
   if (st != MOE_OK) return st;
   const int act = W->act;
-  if (act == MOE_E4M3 && !x_scales) return MOE_ERR_INVALID_ARG;
+  // E4M3 activations without x_scales: x is BF16 and the dispatch quantises it
   const size_t need = moe_workspace_size(MOE_OP_FORWARD, T, H, E, k, I, act, W->wt);
   if (!ws || !aligned(ws, 256) || ws_bytes < need) return MOE_ERR_WORKSPACE;
   const int S = T * k;

@@ -53,12 +53,21 @@ __global__ void __launch_bounds__(256) copy_rows_kernel(
                   threadIdx.x & 31);
 }
 
+// One warp per token: BF16 row -> E4M3 codes + 1x128 scales in each of its k slots.
+__global__ void __launch_bounds__(256) quant_copy_rows_kernel(
+    const __nv_bfloat16* __restrict__ x, int H, const int32_t* __restrict__ slot_of, int T,
+    int k, uint8_t* __restrict__ x_perm, float* __restrict__ x_perm_scales) {
+  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  quant_copy_token_rows(x, H, slot_of, t, k, x_perm, x_perm_scales, threadIdx.x & 31);
+}
+
 }  // namespace
 
 cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes, int T, int H,
                             int E, int k, const int32_t* topk_idx, void* x_perm,
                             float* x_perm_scales, int32_t* offsets, int32_t* perm_src,
-                            int32_t* slot_of, void* ws, cudaStream_t s) {
+                            int32_t* slot_of, void* ws, cudaStream_t s, bool quantize) {
   const int C = (T + kChunkTokens - 1) / kChunkTokens;
   int32_t* cnt = static_cast<int32_t*>(ws);
   const size_t cnt_bytes = ((static_cast<size_t>(C) * E * 4 + 255) / 256) * 256;
@@ -78,9 +87,14 @@ cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes,
   offsets_kernel<<<1, 1024, 0, s>>>(totals, E, offsets);
   slots_kernel<<<blocks, 32 * kWarps, smem, s>>>(topk_idx, T, E, k, C, cnt, offsets, perm_src,
                                                  slot_of);
-  copy_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(static_cast<const uint8_t*>(x), x_scales,
-                                               row_bytes, H / 128, slot_of, T, k,
-                                               static_cast<uint8_t*>(x_perm), x_perm_scales);
+  if (quantize)
+    quant_copy_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(x), H,
+                                                     slot_of, T, k, static_cast<uint8_t*>(x_perm),
+                                                     x_perm_scales);
+  else
+    copy_rows_kernel<<<(T + 7) / 8, 256, 0, s>>>(static_cast<const uint8_t*>(x), x_scales,
+                                                 row_bytes, H / 128, slot_of, T, k,
+                                                 static_cast<uint8_t*>(x_perm), x_perm_scales);
   return cudaGetLastError();
 }
 

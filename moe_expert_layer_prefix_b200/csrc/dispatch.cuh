@@ -187,4 +187,59 @@ __device__ __forceinline__ void copy_token_rows(const uint8_t* __restrict__ x,
   }
 }
 
+// Token t's BF16 row, quantised to E4M3 on the way into its k slots: the activation
+// quantisation that precedes dispatch, fused into the row copy (youleyou, "DeepSeek 模型更新
+// 解读 Tile Kernels 与 DeepEP V2 新特性", Tile Kernels feature list, quantisation item: FP8
+// per-block quantisation; jiqizhixin, "DeepSeek悄悄更新：Mega MoE、FP4 Indexer来了",
+// FP8 x FP4 paragraph: FP8 activations).  Each 1x128 block gets the scale 2^n with n the
+// smallest integer such that amax <= 448 * 2^n (n >= -126; an all-zero block gets 2^0 as
+// the exponent rule gives), codes round to nearest even and saturate: the rule of the h
+// requantisation.  BF16 values are exact in fp32 and the scaling by 2^-n is exact, so the
+// codes depend on the input bits alone.  One warp per token (all 32 lanes call it); lane l
+// holds elements 4l..4l+3 of a block, so loads read 256 contiguous bytes and each slot's
+// codes are written as 128 contiguous bytes per block.
+__device__ __forceinline__ void quant_copy_token_rows(const __nv_bfloat16* __restrict__ x, int H,
+                                                      const int32_t* __restrict__ slot_of, int t,
+                                                      int k, uint8_t* __restrict__ x_perm,
+                                                      float* __restrict__ x_perm_scales,
+                                                      int lane) {
+  constexpr int kB = 4;  // blocks with loads in flight per lane
+  int my_slot = 0;
+  if (lane < k) my_slot = __ldcg(slot_of + static_cast<size_t>(t) * k + lane);
+  int slots[32];
+#pragma unroll
+  for (int j = 0; j < 32; ++j) slots[j] = __shfl_sync(0xffffffffu, my_slot, j);
+  const int nb = H / 128;
+  const uint2* src = reinterpret_cast<const uint2*>(x + static_cast<size_t>(t) * H);
+  for (int b0 = 0; b0 < nb; b0 += kB) {
+    uint2 raw[kB];
+#pragma unroll
+    for (int u = 0; u < kB; ++u)
+      raw[u] = b0 + u < nb ? __ldg(src + static_cast<size_t>(b0 + u) * 32 + lane) : make_uint2(0, 0);
+#pragma unroll
+    for (int u = 0; u < kB; ++u) {
+      if (b0 + u >= nb) break;  // warp-uniform
+      const float2 f01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].x));
+      const float2 f23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[u].y));
+      const float a = fmaxf(fmaxf(fabsf(f01.x), fabsf(f01.y)), fmaxf(fabsf(f23.x), fabsf(f23.y)));
+      // non-negative floats order like their bit patterns
+      const float amax = __uint_as_float(__reduce_max_sync(0xffffffffu, __float_as_uint(a)));
+      const int e = max(e4m3_scale_exponent(amax), -126);
+      const float inv = exp2i(-e);
+      const __nv_fp8x2_storage_t lo =
+          __nv_cvt_float2_to_fp8x2(make_float2(f01.x * inv, f01.y * inv), __NV_SATFINITE, __NV_E4M3);
+      const __nv_fp8x2_storage_t hi =
+          __nv_cvt_float2_to_fp8x2(make_float2(f23.x * inv, f23.y * inv), __NV_SATFINITE, __NV_E4M3);
+      const uint32_t codes = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if (j >= k) break;  // warp-uniform
+        reinterpret_cast<uint32_t*>(x_perm + static_cast<size_t>(slots[j]) * H +
+                                    static_cast<size_t>(b0 + u) * 128)[lane] = codes;
+      }
+      if (lane < k) x_perm_scales[static_cast<size_t>(my_slot) * nb + b0 + u] = exp2i(e);
+    }
+  }
+}
+
 }  // namespace moe

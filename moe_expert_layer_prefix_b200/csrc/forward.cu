@@ -36,6 +36,7 @@ struct FwdParams {
   const float* bias;
   int sigmoid, renorm, T, H, E, k, C;
   int row_bytes;
+  int quant_x;  // x is BF16 and the dispatch quantises it to E4M3 + 1x128 scales
   int32_t* topk_idx;
   float* topk_w;
   int32_t* offsets;
@@ -110,10 +111,16 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
                        lane);
   grid_sync(p.bar, p.err);
 
-  // 6. row copies x -> x_perm (one warp per token)
-  for (int t = gw; t < p.T; t += GW)
-    copy_token_rows(static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes, p.H / 128,
-                    p.slot_of, t, p.k, static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
+  // 6. row copies x -> x_perm (one warp per token), quantising BF16 rows when asked
+  if (p.quant_x) {
+    for (int t = gw; t < p.T; t += GW)
+      quant_copy_token_rows(static_cast<const __nv_bfloat16*>(p.x), p.H, p.slot_of, t, p.k,
+                            static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
+  } else {
+    for (int t = gw; t < p.T; t += GW)
+      copy_token_rows(static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes, p.H / 128,
+                      p.slot_of, t, p.k, static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
+  }
   fence_proxy_async_global();  // x_perm is read by TMA next
   grid_sync(p.bar, p.err);
 
@@ -183,6 +190,7 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   p.k = a.k;
   p.C = (a.T + kChunkTokens - 1) / kChunkTokens;
   p.row_bytes = a.H * (a.act == MOE_BF16 ? 2 : 1);
+  p.quant_x = a.act == MOE_E4M3 && a.x_scales == nullptr;
   p.topk_idx = a.topk_idx;
   p.topk_w = a.topk_w;
   p.offsets = a.offsets;

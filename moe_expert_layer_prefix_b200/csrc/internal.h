@@ -25,7 +25,8 @@ cudaError_t launch_route(const float* logits, const float* bias, int T, int E, i
 cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes, int T, int H,
                             int E, int k, const int32_t* topk_idx, void* x_perm,
                             float* x_perm_scales, int32_t* offsets, int32_t* perm_src,
-                            int32_t* slot_of, void* ws, cudaStream_t s);
+                            int32_t* slot_of, void* ws, cudaStream_t s,
+                            bool quantize = false);
 
 cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, const float* topk_w,
                            int T, int k, int H, void* out, int out_f32, cudaStream_t s);
