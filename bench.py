@@ -17,6 +17,7 @@ sample of the same workload.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import subprocess
@@ -176,6 +177,12 @@ def run_native(args, ws, rank, local):
     M.moe_set_gemm_tiles(args.tiles)
     dev = torch.device("cuda", torch.cuda.current_device())
     d = synth.make_inputs(wl, dev)
+    if args.bf16_input:
+        # BF16 activations into the E4M3 layer: the dispatch quantises them
+        if wl.act != "e4m3":
+            raise SystemExit("--bf16-input needs a workload with E4M3 activations")
+        d["x"] = synth.make_activations(dataclasses.replace(wl, act="bf16"), dev)["x"]
+        d["x_scales"] = None
     W = M.Weights(wl.act, wl.wt, d["w1"], d["w2"], d["w1_scales"], d["w2_scales"])
     T, H, E, k, I, S = wl.T, wl.H, wl.E, wl.k, wl.I, wl.S
     stream = torch.cuda.current_stream()
@@ -183,7 +190,8 @@ def run_native(args, ws, rank, local):
     # buffers of the unfused chain (each call is one C-ABI entry point)
     idx = torch.empty((T, k), dtype=torch.int32, device=dev)
     gw = torch.empty((T, k), dtype=torch.float32, device=dev)
-    disp = {"x_perm": torch.empty((S, H), dtype=d["x"].dtype, device=dev),
+    xdt = {"f32": torch.float32, "bf16": torch.bfloat16, "e4m3": torch.uint8}[wl.act]
+    disp = {"x_perm": torch.empty((S, H), dtype=xdt, device=dev),
             "x_perm_scales": (torch.empty((S, H // 128), dtype=torch.float32, device=dev)
                               if wl.act == "e4m3" else None),
             "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
@@ -207,8 +215,11 @@ def run_native(args, ws, rank, local):
         M.moe_route(d["logits"], k, wl.score, bias=d["bias"], renorm=wl.renorm, topk_idx=idx,
                     topk_w=gw, stream=stream)
         mark(1)
-        M.moe_dispatch(d["x"], idx, E, wl.act, x_scales=d["x_scales"], ws=dws, out=disp,
-                       stream=stream)
+        if args.bf16_input:
+            M.moe_dispatch_quant(d["x"], idx, E, ws=dws, out=disp, stream=stream)
+        else:
+            M.moe_dispatch(d["x"], idx, E, wl.act, x_scales=d["x_scales"], ws=dws, out=disp,
+                           stream=stream)
         mark(2)
         M.moe_expert_linear1(disp["x_perm"], disp["expert_offsets"], W,
                              x_perm_scales=disp["x_perm_scales"], h=h, h_scales=hs,
@@ -384,6 +395,8 @@ def run_native(args, ws, rank, local):
         "data": "synthetic (seeded; random-init weights of the workload's shape)",
         "config": {"workload": wl.name, "T": T, "H": H, "E": E, "k": k, "I": I, "act": wl.act,
                    "wt": wl.wt, "router": wl.score, "experts_touched": touched,
+                   "input": ("bf16, quantised to e4m3 in the dispatch" if args.bf16_input
+                             else wl.act),
                    "l2": "inputs larger than L2 (expert weights >> 126 MB), no flush",
                    "parallelism": f"replicas x{ws}"},
         "tflops": wl.flops() / (ms / 1e3) / 1e12 * ws,
@@ -485,6 +498,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="v3_fp8", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--bf16-input", action="store_true",
+                    help="E4M3 workloads: feed BF16 activations, quantised in the dispatch")
     ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair", "small"],
                     help="tile shape of the expert GEMMs")
     ap.add_argument("--T", type=int, default=None, help="override T (profiling captures)")

@@ -263,19 +263,20 @@ def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=Tru
     return out
 
 
-def moe_dispatch_quant(x, topk_idx, E, ws=None, stream=None):
+def moe_dispatch_quant(x, topk_idx, E, ws=None, out=None, stream=None):
     """Dispatch of BF16 rows x [T, H] into an E4M3 layer, quantising on the way (1x128
     power-of-two scales).  Returns dict(x_perm (E4M3 codes, uint8), x_perm_scales,
-    expert_offsets, perm_src, slot_of)."""
+    expert_offsets, perm_src, slot_of); tensors given in `out` are written in place."""
     T, H = x.shape
     k = topk_idx.shape[1]
     S = T * k
     dev = x.device
-    r = {"x_perm": torch.empty((S, H), dtype=torch.uint8, device=dev),
-         "x_perm_scales": torch.empty((S, H // 128), dtype=torch.float32, device=dev),
-         "expert_offsets": torch.empty(E + 1, dtype=torch.int32, device=dev),
-         "perm_src": torch.empty(S, dtype=torch.int32, device=dev),
-         "slot_of": torch.empty(S, dtype=torch.int32, device=dev)}
+    o = out or {}
+    shapes = {"x_perm": ((S, H), torch.uint8), "x_perm_scales": ((S, H // 128), torch.float32),
+              "expert_offsets": ((E + 1,), torch.int32), "perm_src": ((S,), torch.int32),
+              "slot_of": ((S,), torch.int32)}
+    r = {key: (o[key] if o.get(key) is not None else torch.empty(shp, dtype=dt, device=dev))
+         for key, (shp, dt) in shapes.items()}
     need = moe_workspace_size("dispatch", T, H, E, k, 128, "e4m3", "e4m3")
     if ws is None:
         ws = workspace(need, dev)
