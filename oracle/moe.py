@@ -44,13 +44,19 @@ E4M3_MAX = 448.0
 # ----------------------------------------------------------------------------------------
 # 1. route
 # ----------------------------------------------------------------------------------------
-def route(logits, bias, k: int, score: str, renorm: bool = True):
+def route(logits, bias, k: int, score: str, renorm: bool = True, n_group: int = 1,
+          topk_group: int = 0, scale: float = 1.0):
     """Top-k expert selection and gate weights.
 
     softmax: keys are the fp32 logits themselves; gates are exp(l_j - m) / sum over the k
              selected (renorm) or over all E experts (no renorm), m the largest logit used.
     sigmoid: s = sigmoid(l) in fp32 (oracle.fexp), keys = fp32(s + b_e); gates are
              s_j / sum of the selected s (renorm) or s_j (no renorm).
+    Group-limited selection (n_group > 1): experts form n_group consecutive groups of
+    E / n_group; a group's score is the fp32 sum of its two largest keys (its only key when
+    a group holds one expert); the topk_group best groups (equal scores -> lower group id)
+    are kept and the k experts are chosen among theirs only.  Gates are finally multiplied
+    by `scale` (the routed scaling factor; 1 leaves them as they are).
     Order: key descending, equal keys -> lower expert id first.  The k experts are returned
     in that rank order, which is also the order in which the combine sums them.
 
@@ -65,10 +71,21 @@ def route(logits, bias, k: int, score: str, renorm: bool = True):
         keys = (s + b[None, :]).astype(np.float32)
     else:
         raise ValueError(score)
-    # a stable sort of the negated keys keeps equal keys in ascending expert order
-    order = np.argsort(-keys, axis=1, kind="stable")
-    idx = order[:, :k].astype(np.int32)
     rows = np.arange(T)[:, None]
+    ids = np.broadcast_to(np.arange(E), (T, E))
+    if n_group > 1:
+        G = E // n_group
+        srt = np.sort(keys.reshape(T, n_group, G), axis=2)
+        gscore = srt[:, :, -1] if G == 1 else (srt[:, :, -1] + srt[:, :, -2]).astype(np.float32)
+        gorder = np.argsort(-gscore, axis=1, kind="stable")[:, :topk_group]
+        allowed = np.zeros((T, n_group), bool)
+        allowed[rows, gorder] = True
+        allowed = np.repeat(allowed, G, axis=1)
+    else:
+        allowed = np.ones((T, E), bool)
+    # allowed experts first, then key descending, then expert id ascending
+    order = np.lexsort((ids, -keys, ~allowed), axis=1)
+    idx = order[:, :k].astype(np.int32)
     if score == "softmax":
         l = logits.astype(np.float64)
         sel = l[rows, idx]
@@ -81,7 +98,7 @@ def route(logits, bias, k: int, score: str, renorm: bool = True):
     else:
         ssel = s.astype(np.float64)[rows, idx]
         w = ssel / ssel.sum(axis=1, keepdims=True) if renorm else ssel
-    return idx, w
+    return idx, w * scale
 
 
 # ----------------------------------------------------------------------------------------

@@ -308,3 +308,57 @@ def test_synth_e4m3_decodes_like_torch():
         .repeat_interleave(128, 1)
     got = oracle.dequant_x(d["x"].numpy(), d["x_scales"].numpy(), "e4m3")
     assert np.array_equal(ref.numpy(), got)
+
+
+# ----------------------------------------------------------------------- group-limited routing
+def _route_grouped_brute(keys, k, n_group, topk_group):
+    """Plain-Python restatement: group score = sum of a group's two largest keys (fp32 add),
+    keep the topk_group best groups (ties -> lower group), then the k best experts of the
+    kept groups (ties -> lower expert)."""
+    T, E = keys.shape
+    G = E // n_group
+    out = []
+    for t in range(T):
+        gs = []
+        for g in range(n_group):
+            ks = sorted((float(keys[t, e]) for e in range(g * G, (g + 1) * G)), reverse=True)
+            sc = ks[0] if G == 1 else float(np.float32(ks[0]) + np.float32(ks[1]))
+            gs.append((-sc, g))
+        kept = {g for _, g in sorted(gs)[:topk_group]}
+        cand = sorted((-float(keys[t, e]), e) for e in range(E) if e // G in kept)
+        out.append([e for _, e in cand[:k]])
+    return np.array(out, np.int32)
+
+
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+@pytest.mark.parametrize("E,n_group,topk_group,k", [(16, 4, 2, 3), (32, 8, 3, 4), (12, 12, 5, 5),
+                                                    (64, 2, 1, 8)])
+def test_route_grouped_brute_force(score, E, n_group, topk_group, k):
+    rng = np.random.default_rng(E + n_group)
+    logits = rng.standard_normal((40, E)).astype(np.float32)
+    logits[::5] = np.round(logits[::5])            # many equal keys and group scores
+    bias = (rng.standard_normal(E) * 0.1).astype(np.float32)
+    idx, _ = oracle.route(logits, bias if score == "sigmoid" else None, k, score,
+                          n_group=n_group, topk_group=topk_group)
+    keys = logits if score == "softmax" else (oracle.sigmoid_f32(logits) + bias).astype(np.float32)
+    assert np.array_equal(idx, _route_grouped_brute(keys, k, n_group, topk_group))
+
+
+def test_route_grouped_all_groups_is_plain_routing_and_scale_multiplies():
+    rng = np.random.default_rng(3)
+    logits = rng.standard_normal((20, 64)).astype(np.float32)
+    bias = (rng.standard_normal(64) * 0.1).astype(np.float32)
+    for score in ("softmax", "sigmoid"):
+        b = bias if score == "sigmoid" else None
+        i0, w0 = oracle.route(logits, b, 6, score)
+        i1, w1 = oracle.route(logits, b, 6, score, n_group=8, topk_group=8, scale=2.5)
+        assert np.array_equal(i0, i1)
+        assert np.array_equal(w0 * 2.5, w1)
+
+
+def test_route_grouped_excludes_a_strong_expert_in_a_weak_group():
+    # group 0 holds the single best expert but a weak second; groups 1 and 2 are stronger
+    # by their top-2 sums, so with topk_group = 2 expert 0 must not be chosen
+    keys = np.array([[5.0, -9, -9, -9, 3, 3, -9, -9, 2.9, 2.9, -9, -9]], np.float32)
+    idx, _ = oracle.route(keys, None, 2, "softmax", n_group=3, topk_group=2)
+    assert idx.tolist() == [[4, 5]]
