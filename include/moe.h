@@ -94,6 +94,29 @@ typedef struct moe_weights {
 moe_status moe_route(const float* logits, const float* bias, int T, int E, int k, int score,
                      int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t stream);
 
+/* Group-limited routing and the routed scaling factor, for moe_route_ex / moe_forward_ex.
+ * The experts form n_group consecutive groups of G = E / n_group (G a multiple of 32, or
+ * n_group = 1).  A group's score is the fp32 sum of its two largest selection keys (as
+ * moe_route forms them); the topk_group best groups (equal scores -> lower group) are kept
+ * and the k experts are selected among theirs only, in the same rank order.  The gates are
+ * then multiplied by `scale`.  {1, 1, 1.0f} is moe_route itself.  Not on the source pages,
+ * which only name gating with top-k selection and weight normalisation; this is the
+ * DeepSeek-V3-style variant of it.
+ *   errors: MOE_ERR_INVALID_ARG for n_group < 1, topk_group outside [1, n_group],
+ *           k > topk_group * G or a non-finite scale; MOE_ERR_UNSUPPORTED when E is not a
+ *           multiple of n_group or G is not a multiple of 32 (n_group > 1). */
+typedef struct {
+  int n_group;
+  int topk_group;
+  float scale;
+} moe_router_groups;
+
+/* moe_route with group-limited selection and a routed scaling factor (groups may be NULL:
+ * moe_route). */
+moe_status moe_route_ex(const float* logits, const float* bias, int T, int E, int k, int score,
+                        int renorm, const moe_router_groups* groups, int32_t* topk_idx,
+                        float* topk_w, cudaStream_t stream);
+
 /* Dispatch: permute token rows to experts (stable counting sort by expert).
  * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: tokens are dispatched to the
  *  experts; youleyou, routing item: token-to-expert mapping with fused expand.)
@@ -182,6 +205,14 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
                        int I, const moe_weights* W, void* out, int32_t* topk_idx,
                        float* topk_w, int32_t* expert_offsets, void* ws, size_t ws_bytes,
                        cudaStream_t stream);
+
+/* moe_forward routed as moe_route_ex does (groups may be NULL: moe_forward). */
+moe_status moe_forward_ex(const void* x, const float* x_scales, const float* logits,
+                          const float* bias, int score, int renorm,
+                          const moe_router_groups* groups, int T, int H, int E, int k, int I,
+                          const moe_weights* W, void* out, int32_t* topk_idx, float* topk_w,
+                          int32_t* expert_offsets, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
 
 /* moe_dispatch without a caller workspace, for callers that cannot allocate device memory
  * (a host with no device allocator of its own, a runtime that forbids allocations after

@@ -34,9 +34,14 @@ OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5}
 EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
            "moe_get_device_error", "moe_status_string", "moe_launch_count",
-           "moe_dispatch_noalloc", "moe_set_gemm_tiles", "moe_dispatch_quant")
+           "moe_dispatch_noalloc", "moe_set_gemm_tiles", "moe_dispatch_quant", "moe_route_ex",
+           "moe_forward_ex")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+
+
+class MoeRouterGroups(ctypes.Structure):
+    _fields_ = [("n_group", ctypes.c_int), ("topk_group", ctypes.c_int), ("scale", ctypes.c_float)]
 
 
 class MoeWeights(ctypes.Structure):
@@ -51,6 +56,8 @@ def _sig(name, res, args):
 
 
 _route = _sig("moe_route", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P])
+_route_ex = _sig("moe_route_ex", _I, [_P, _P, _I, _I, _I, _I, _I, ctypes.POINTER(MoeRouterGroups),
+                                      _P, _P, _P])
 _dispatch = _sig("moe_dispatch", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P, _Z,
                                       _P])
 _linear1 = _sig("moe_expert_linear1", _I, [_P, _P, _P, _I, _I, _I, _I,
@@ -66,6 +73,9 @@ _dispatch_quant = _sig("moe_dispatch_quant", _I, [_P, _I, _I, _I, _I, _P, _P, _P
 _combine = _sig("moe_combine", _I, [_P, _I, _P, _P, _I, _I, _I, _P, _I, _P])
 _forward = _sig("moe_forward", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                     ctypes.POINTER(MoeWeights), _P, _P, _P, _P, _P, _Z, _P])
+_forward_ex = _sig("moe_forward_ex", _I, [_P, _P, _P, _P, _I, _I, ctypes.POINTER(MoeRouterGroups),
+                                          _I, _I, _I, _I, _I, ctypes.POINTER(MoeWeights), _P, _P,
+                                          _P, _P, _P, _Z, _P])
 _ws_size = _sig("moe_workspace_size", _Z, [_I, _I, _I, _I, _I, _I, _I, _I])
 _get_err = _sig("moe_get_device_error", _I, [_P, ctypes.POINTER(ctypes.c_int)])
 _status_string = _sig("moe_status_string", ctypes.c_char_p, [_I])
@@ -145,15 +155,29 @@ class Weights:
                             None if w2_scales is None else w2_scales.data_ptr())
 
 
+def _groups(groups):
+    """(n_group, topk_group, scale) -> a moe_router_groups the call can point at."""
+    n_group, topk_group, scale = groups
+    return MoeRouterGroups(int(n_group), int(topk_group), float(scale))
+
+
 def moe_route(logits, k, score="softmax", bias=None, renorm=True, topk_idx=None, topk_w=None,
-              stream=None):
+              stream=None, groups=None):
+    """Top-k routing.  groups=(n_group, topk_group, scale) selects group-limited routing with
+    a routed scaling factor (moe_route_ex)."""
     T, E = logits.shape
     if topk_idx is None:
         topk_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=logits.device)
-    _check(_route(_ptr(logits), _ptr(bias), T, E, k, SCORES[score], int(renorm), _ptr(topk_idx),
-                  _ptr(topk_w), _stream(stream)), "moe_route")
+    if groups is None:
+        _check(_route(_ptr(logits), _ptr(bias), T, E, k, SCORES[score], int(renorm),
+                      _ptr(topk_idx), _ptr(topk_w), _stream(stream)), "moe_route")
+    else:
+        g = _groups(groups)
+        _check(_route_ex(_ptr(logits), _ptr(bias), T, E, k, SCORES[score], int(renorm),
+                         ctypes.byref(g), _ptr(topk_idx), _ptr(topk_w), _stream(stream)),
+               "moe_route_ex")
     return topk_idx, topk_w
 
 
@@ -244,9 +268,10 @@ def moe_combine(y, slot_of, topk_w, out=None, out_dtype=None, stream=None):
 
 def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=True,
                 x_scales=None, out=None, ws=None, topk_idx=None, topk_w=None,
-                expert_offsets=None, stream=None):
+                expert_offsets=None, stream=None, groups=None):
     """The whole layer.  For an E4M3 layer, x is either E4M3 codes with x_scales, or BF16 with
-    x_scales=None (quantised by the dispatch)."""
+    x_scales=None (quantised by the dispatch).  groups=(n_group, topk_group, scale) routes as
+    moe_route does with the same argument (moe_forward_ex)."""
     T, H = x.shape
     E = logits.shape[1]
     dev = x.device
@@ -256,10 +281,17 @@ def moe_forward(x, logits, W: Weights, k, score="softmax", bias=None, renorm=Tru
     need = moe_workspace_size("forward", T, H, E, k, W.I, W.act, W.wt)
     if ws is None:
         ws = workspace(need, dev)
-    _check(_forward(_ptr(x), _ptr(x_scales), _ptr(logits), _ptr(bias), SCORES[score],
-                    int(renorm), T, H, E, k, W.I, ctypes.byref(W.c), _ptr(out), _ptr(topk_idx),
-                    _ptr(topk_w), _ptr(expert_offsets), _ptr(ws), ws.numel(), _stream(stream)),
-           "moe_forward")
+    if groups is None:
+        _check(_forward(_ptr(x), _ptr(x_scales), _ptr(logits), _ptr(bias), SCORES[score],
+                        int(renorm), T, H, E, k, W.I, ctypes.byref(W.c), _ptr(out),
+                        _ptr(topk_idx), _ptr(topk_w), _ptr(expert_offsets), _ptr(ws), ws.numel(),
+                        _stream(stream)), "moe_forward")
+    else:
+        g = _groups(groups)
+        _check(_forward_ex(_ptr(x), _ptr(x_scales), _ptr(logits), _ptr(bias), SCORES[score],
+                           int(renorm), ctypes.byref(g), T, H, E, k, W.I, ctypes.byref(W.c),
+                           _ptr(out), _ptr(topk_idx), _ptr(topk_w), _ptr(expert_offsets),
+                           _ptr(ws), ws.numel(), _stream(stream)), "moe_forward_ex")
     return out
 
 

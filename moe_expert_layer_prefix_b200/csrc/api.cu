@@ -182,8 +182,29 @@ moe_status moe_get_device_error(cudaStream_t stream, int* site) {
   return static_cast<moe_status>(host[0]);
 }
 
+// Checks a routing configuration; fills in the plain router for NULL.
+static moe_status check_groups(const moe_router_groups* g, int E, int k, moe_router_groups* out) {
+  *out = moe_router_groups{1, 1, 1.0f};
+  if (g == nullptr) return MOE_OK;
+  if (g->n_group < 1 || g->topk_group < 1 || g->topk_group > g->n_group) return MOE_ERR_INVALID_ARG;
+  if (!(g->scale == g->scale) || g->scale == INFINITY || g->scale == -INFINITY)
+    return MOE_ERR_INVALID_ARG;
+  if (g->n_group > 1) {
+    if (E % g->n_group != 0 || (E / g->n_group) % 32 != 0) return MOE_ERR_UNSUPPORTED;
+    if (k > g->topk_group * (E / g->n_group)) return MOE_ERR_INVALID_ARG;
+  }
+  *out = *g;
+  return MOE_OK;
+}
+
 moe_status moe_route(const float* logits, const float* bias, int T, int E, int k, int score,
                      int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t stream) {
+  return moe_route_ex(logits, bias, T, E, k, score, renorm, nullptr, topk_idx, topk_w, stream);
+}
+
+moe_status moe_route_ex(const float* logits, const float* bias, int T, int E, int k, int score,
+                        int renorm, const moe_router_groups* groups, int32_t* topk_idx,
+                        float* topk_w, cudaStream_t stream) {
   if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 1 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
   if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
@@ -191,8 +212,12 @@ moe_status moe_route(const float* logits, const float* bias, int T, int E, int k
   if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
       (bias && !aligned(bias, 4)))
     return MOE_ERR_MISALIGNED;
+  moe_router_groups g;
+  const moe_status gs = check_groups(groups, E, k, &g);
+  if (gs != MOE_OK) return gs;
   return cuda_status(launch_route(logits, score == MOE_SCORE_SIGMOID ? bias : nullptr, T, E, k,
-                                  score, renorm != 0, topk_idx, topk_w, stream));
+                                  score, renorm != 0, topk_idx, topk_w, stream, g.n_group,
+                                  g.topk_group, g.scale));
 }
 
 moe_status moe_dispatch(const void* x, const float* x_scales, int act, int T, int H, int E, int k,
@@ -309,7 +334,20 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
                        int I, const moe_weights* W, void* out, int32_t* topk_idx_out,
                        float* topk_w_out, int32_t* offsets_out, void* ws, size_t ws_bytes,
                        cudaStream_t stream) {
+  return moe_forward_ex(x, x_scales, logits, bias, score, renorm, nullptr, T, H, E, k, I, W, out,
+                        topk_idx_out, topk_w_out, offsets_out, ws, ws_bytes, stream);
+}
+
+moe_status moe_forward_ex(const void* x, const float* x_scales, const float* logits,
+                          const float* bias, int score, int renorm,
+                          const moe_router_groups* groups, int T, int H, int E, int k, int I,
+                          const moe_weights* W, void* out, int32_t* topk_idx_out,
+                          float* topk_w_out, int32_t* offsets_out, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
   moe_status st = check_shapes(T, H, E, k);
+  if (st != MOE_OK) return st;
+  moe_router_groups rg;
+  st = check_groups(groups, E, k, &rg);
   if (st != MOE_OK) return st;
   if (I < 128) return MOE_ERR_INVALID_ARG;
   if (I % 128 != 0) return MOE_ERR_UNSUPPORTED;
@@ -358,6 +396,9 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
     fa.bias = score == MOE_SCORE_SIGMOID ? bias : nullptr;
     fa.sigmoid = score == MOE_SCORE_SIGMOID;
     fa.renorm = renorm != 0;
+    fa.n_group = rg.n_group;
+    fa.topk_group = rg.topk_group;
+    fa.scale = rg.scale;
     fa.T = T;
     fa.H = H;
     fa.E = E;
@@ -388,7 +429,7 @@ moe_status moe_forward(const void* x, const float* x_scales, const float* logits
     return cuda_status(launch_forward_fused(fa, stream));
   }
 
-  st = moe_route(logits, bias, T, E, k, score, renorm, topk_idx, topk_w, stream);
+  st = moe_route_ex(logits, bias, T, E, k, score, renorm, &rg, topk_idx, topk_w, stream);
   if (st != MOE_OK) return st;
   st = moe_dispatch(x, x_scales, act, T, H, E, k, topk_idx, x_perm, x_perm_scales, offsets,
                     perm_src, slot_of, dws, dispatch_ws_bytes(T, E), stream);

@@ -37,6 +37,8 @@ struct FwdParams {
   int sigmoid, renorm, T, H, E, k, C;
   int row_bytes;
   int quant_x;  // x is BF16 and the dispatch quantises it to E4M3 + 1x128 scales
+  int n_group, topk_group;
+  float scale;
   int32_t* topk_idx;
   float* topk_w;
   int32_t* offsets;
@@ -84,10 +86,12 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   // 1. route: one warp per token
   if (p.E <= 256) {
     for (int t = gw; t < p.T; t += GW)
-      route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+      route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
+                     p.n_group, p.topk_group, p.scale);
   } else {
     for (int t = gw; t < p.T; t += GW)
-      route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane);
+      route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
+                      p.n_group, p.topk_group, p.scale);
   }
   grid_sync(p.bar, p.err);
 
@@ -184,6 +188,9 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   p.bias = a.bias;
   p.sigmoid = a.sigmoid;
   p.renorm = a.renorm;
+  p.n_group = a.n_group;
+  p.topk_group = a.topk_group;
+  p.scale = a.scale;
   p.T = a.T;
   p.H = a.H;
   p.E = a.E;

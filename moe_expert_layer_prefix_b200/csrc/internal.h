@@ -20,7 +20,8 @@ inline size_t dispatch_ws_bytes(int T, int E) {
 }
 
 cudaError_t launch_route(const float* logits, const float* bias, int T, int E, int k, int score,
-                         int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s);
+                         int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s,
+                         int n_group = 1, int topk_group = 1, float scale = 1.0f);
 
 cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes, int T, int H,
                             int E, int k, const int32_t* topk_idx, void* x_perm,
@@ -64,6 +65,8 @@ struct ForwardArgs {
   const float* logits;
   const float* bias;
   int sigmoid, renorm, T, H, E, k, I;
+  int n_group = 1, topk_group = 1;  // group-limited routing (1, 1: plain)
+  float scale = 1.0f;               // routed scaling factor
   int act, wt;
   const void* w1;
   const void* w1_scales;

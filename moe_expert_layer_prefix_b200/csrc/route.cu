@@ -12,33 +12,34 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     const float* __restrict__ bias, int T, int E,
                                                     int k, int sigmoid, int renorm,
                                                     int32_t* __restrict__ topk_idx,
-                                                    float* __restrict__ topk_w) {
+                                                    float* __restrict__ topk_w, int n_group,
+                                                    int topk_group, float scale) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (t >= T) return;
-  route_token<NPL>(logits, bias, t, E, k, sigmoid, renorm, topk_idx, topk_w, threadIdx.x & 31);
+  route_token<NPL>(logits, bias, t, E, k, sigmoid, renorm, topk_idx, topk_w, threadIdx.x & 31,
+                   n_group, topk_group, scale);
 }
 
 }  // namespace
 
 cudaError_t launch_route(const float* logits, const float* bias, int T, int E, int k, int score,
-                         int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s) {
+                         int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s,
+                         int n_group, int topk_group, float scale) {
   const int warps = 8;
   dim3 grid((T + warps - 1) / warps), block(32 * warps);
   const int sig = score == MOE_SCORE_SIGMOID;
   const int npl = (E + 31) / 32;
   count_launch();
-  if (npl <= 1)
-    route_kernel<1><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
-  else if (npl <= 2)
-    route_kernel<2><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
-  else if (npl <= 4)
-    route_kernel<4><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
-  else if (npl <= 8)
-    route_kernel<8><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
-  else if (npl <= 16)
-    route_kernel<16><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
-  else
-    route_kernel<32><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w);
+#define MOE_ROUTE(N)                                                                        \
+  route_kernel<N><<<grid, block, 0, s>>>(logits, bias, T, E, k, sig, renorm, topk_idx, topk_w, \
+                                         n_group, topk_group, scale)
+  if (npl <= 1) MOE_ROUTE(1);
+  else if (npl <= 2) MOE_ROUTE(2);
+  else if (npl <= 4) MOE_ROUTE(4);
+  else if (npl <= 8) MOE_ROUTE(8);
+  else if (npl <= 16) MOE_ROUTE(16);
+  else MOE_ROUTE(32);
+#undef MOE_ROUTE
   return cudaGetLastError();
 }
 

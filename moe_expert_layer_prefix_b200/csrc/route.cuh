@@ -54,12 +54,19 @@ __device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
 
 // One warp selects the k experts of token t and writes topk_idx[t, :], topk_w[t, :].
 // Lanes hold experts lane, lane+32, ...; all 32 lanes must call it together.
+// Group-limited selection (n_group > 1, groups of G = E / n_group experts with G a multiple
+// of 32): a group's score is the fp32 sum of its two largest keys, the topk_group best groups
+// (equal scores -> lower group) are kept and the k experts are chosen among theirs only.
+// Gates are multiplied by `scale` (the routed scaling factor).  n_group = 1, scale = 1 is
+// the plain router.
 template <int NPL>  // experts per lane (E <= 32 * NPL)
 __device__ __forceinline__ void route_token(const float* __restrict__ logits,
                                             const float* __restrict__ bias, int t, int E, int k,
                                             int sigmoid, int renorm,
                                             int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_w, int lane) {
+                                            float* __restrict__ topk_w, int lane,
+                                            int n_group = 1, int topk_group = 1,
+                                            float scale = 1.0f) {
   const float* row = logits + static_cast<size_t>(t) * E;
 
   float key[NPL];
@@ -94,7 +101,56 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
     u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
     return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~e);
   };
+  // Groups.  Lane l holds experts l + 32i, so with G a multiple of 32 a group is sg = G / 32
+  // consecutive slots i of every lane: each lane keeps a running top-2 over the group's
+  // slots and the warp merges them at the group's last slot; slots of groups that are not
+  // kept start out as taken.
   uint32_t taken = 0;
+  if (n_group > 1) {
+    const int sg = E / n_group / 32;
+    float gsc[NPL];    // at a group's last slot: the group's score
+    float a1 = -INFINITY, a2 = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      gsc[i] = -INFINITY;
+      if (32 * i < E) {
+        const float x = key[i];
+        a2 = fmaxf(a2, fminf(a1, x));
+        a1 = fmaxf(a1, x);
+        if ((i + 1) % sg == 0) {  // warp-uniform
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) {
+            const float b1v = __shfl_xor_sync(0xffffffffu, a1, off);
+            const float b2v = __shfl_xor_sync(0xffffffffu, a2, off);
+            const float hi = fmaxf(a1, b1v);
+            a2 = fmaxf(fminf(a1, b1v), fmaxf(a2, b2v));
+            a1 = hi;
+          }
+          gsc[i] = __fadd_rn(a1, a2);
+          a1 = a2 = -INFINITY;
+        }
+      }
+    }
+    uint32_t keep = 0;  // bit i: slot i is the last slot of a kept group
+    for (int r = 0; r < topk_group; ++r) {
+      float best = 0.0f;
+      int bi = -1;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        if (32 * i < E && (i + 1) % sg == 0 && !((keep >> i) & 1u) &&
+            (bi < 0 || gsc[i] > best)) {
+          best = gsc[i];
+          bi = i;
+        }
+      }
+      if (bi >= 0) keep |= 1u << bi;
+    }
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) {
+      const int last = (i / sg) * sg + sg - 1;
+      if (!((keep >> last) & 1u)) taken |= 1u << i;
+    }
+  }
   uint64_t b1 = 0, b2 = 0;  // this lane's best and second-best untaken candidates
   float v1 = 0.0f, v2 = 0.0f;
   auto scan = [&]() {
@@ -178,7 +234,7 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
   }
   if (lane < k) {
     topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
-    topk_w[static_cast<size_t>(t) * k + lane] = g;
+    topk_w[static_cast<size_t>(t) * k + lane] = g * scale;
   }
 }
 
