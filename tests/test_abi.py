@@ -47,3 +47,35 @@ def test_workspace_sizes():
     assert M.moe_workspace_size("forward", T, H, E, k, I, "bf16", "e4m3") == 0
     assert M.moe_workspace_size(99, T, H, E, k, I, "e4m3", "e4m3") == 0
     assert M.moe_workspace_size("forward", 0, H, E, k, I, "e4m3", "e4m3") == 0
+
+
+def test_tile_shape_knob_accepts_the_documented_values_only():
+    # host-side setting (no launch): 0 auto, 1 single, 2 pair, 3 small
+    try:
+        for mode in ("auto", "single", "pair", "small", 0, 1, 2, 3):
+            M.moe_set_gemm_tiles(mode)
+        for bad in (-1, 4):
+            try:
+                M.moe_set_gemm_tiles(bad)
+            except M.MoeError as e:
+                assert "MOE_ERR_INVALID_ARG" in str(e)
+            else:
+                raise AssertionError(f"mode {bad} accepted")
+    finally:
+        M.moe_set_gemm_tiles("auto")
+
+
+def test_argument_errors_need_no_gpu():
+    # argument checks run before anything touches a device, so they work on a host alone
+    P = None
+    st = M._route_ex(P, P, 4, 256, 8, 0, 1, None, P, P, P)
+    assert M.moe_status_string(st) == "MOE_ERR_INVALID_ARG"            # NULL logits
+    st = M._dispatch_quant(P, 4, 256, 8, 2, P, P, P, P, P, P, P, 0, P)
+    assert M.moe_status_string(st) == "MOE_ERR_INVALID_ARG"            # NULL buffers
+    # a group configuration the GPU router does not take is refused before any launch (the
+    # aligned dummy addresses are never dereferenced)
+    import ctypes
+    fake = ctypes.c_void_p(1 << 20)
+    g = M.MoeRouterGroups(3, 1, 1.0)                                  # 256 experts / 3 groups
+    st = M._route_ex(fake, None, 4, 256, 8, 0, 1, ctypes.byref(g), fake, fake, None)
+    assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
