@@ -93,9 +93,9 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
   // Selection.  A candidate is packed into one 64-bit word ordered like (key, id): the key
   // as an order-preserving integer in the high half (-0 taken as +0, so that equal keys give
   // equal words), the complemented id in the low half (lower id wins a tie).  0 is below
-  // every candidate.  Each lane caches its best two untaken candidates; a round takes the
-  // warp maximum of the lanes' best (5 shuffle steps), the winning lane moves its second
-  // up, and only a lane that wins twice in a row rescans its NPL experts.
+  // every candidate.  Each lane caches its best four untaken candidates; a round takes the
+  // warp maximum of the lanes' best (5 shuffle steps), the winning lane moves its list up,
+  // and only a lane whose four are all taken rescans its NPL experts.
   auto pack = [](float key, int e) -> uint64_t {
     uint32_t u = __float_as_uint(__fadd_rn(key, 0.0f));
     u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -151,34 +151,50 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
       if (!((keep >> last) & 1u)) taken |= 1u << i;
     }
   }
-  uint64_t b1 = 0, b2 = 0;  // this lane's best and second-best untaken candidates
-  float v1 = 0.0f, v2 = 0.0f;
+  // This lane's best four untaken candidates in order (c[0] best; 0 = none) and their
+  // values; the winning lane shifts its list up and rescans only once all four are gone.
+  constexpr int kC = 4;
+  uint64_t c[kC];
+  float cv[kC];
+  int n_c = 0;  // valid entries of c
   auto scan = [&]() {
-    b1 = b2 = 0;
+#pragma unroll
+    for (int q = 0; q < kC; ++q) {
+      c[q] = 0;
+      cv[q] = 0.0f;
+    }
 #pragma unroll
     for (int i = 0; i < NPL; ++i) {
       const int e = lane + 32 * i;
       if (e < E && !((taken >> i) & 1u)) {
-        const uint64_t c = pack(key[i], e);
-        if (c > b1) {
-          b2 = b1;
-          v2 = v1;
-          b1 = c;
-          v1 = val[i];
-        } else if (c > b2) {
-          b2 = c;
-          v2 = val[i];
+        const uint64_t x = pack(key[i], e);
+        if (x > c[kC - 1]) {  // insert, keeping c sorted
+          uint64_t y = x;
+          float yv = val[i];
+#pragma unroll
+          for (int q = 0; q < kC; ++q) {
+            if (y > c[q]) {
+              const uint64_t t0 = c[q];
+              const float tv = cv[q];
+              c[q] = y;
+              cv[q] = yv;
+              y = t0;
+              yv = tv;
+            }
+          }
         }
       }
     }
+    n_c = 0;
+#pragma unroll
+    for (int q = 0; q < kC; ++q) n_c += c[q] != 0;
   };
   scan();
-  bool second_ok = true;  // b2 is this lane's true second best
   int my_idx = 0;      // lane j keeps the j-th selection
   float my_val = 0.0f;
   float top_val = 0.0f;
   for (int j = 0; j < k; ++j) {
-    uint64_t best = b1;
+    uint64_t best = c[0];
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
       const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
@@ -186,17 +202,19 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
     }
     const int bi = static_cast<int>(~static_cast<uint32_t>(best));
     const int owner = bi & 31;
-    const float bv = __shfl_sync(0xffffffffu, v1, owner);
+    const float bv = __shfl_sync(0xffffffffu, cv[0], owner);
     if (lane == owner) {
       taken |= 1u << (bi >> 5);
-      if (second_ok) {
-        b1 = b2;
-        v1 = v2;
-        b2 = 0;
-        second_ok = false;
+      if (n_c > 1) {
+#pragma unroll
+        for (int q = 0; q + 1 < kC; ++q) {
+          c[q] = c[q + 1];
+          cv[q] = cv[q + 1];
+        }
+        c[kC - 1] = 0;
+        --n_c;
       } else {
         scan();
-        second_ok = true;
       }
     }
     if (lane == j) {
