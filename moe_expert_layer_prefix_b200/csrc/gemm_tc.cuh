@@ -29,7 +29,8 @@
 //               (leader's) slot barriers; before each GEMM phase it also builds the tile list
 //   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp i reads TMEM lanes 32i..32i+31,
 //               one output row per thread), SwiGLU + BF16 / E4M3 requantisation (linear-1)
-//               or BF16 conversion (linear-2), 16-byte global stores
+//               or BF16 conversion (linear-2); 16-byte global stores, for linear-2 after
+//               lane pairs swap chunks so that every store writes whole 32-byte sectors
 //
 // linear-1 tiles take B rows [n*128, n*128+128) (gate) and [I + n*128, ...) (up), so the
 // accumulator holds gate in columns 0..127 and up in 128..255 and each tile yields 128 h
@@ -62,8 +63,8 @@ constexpr int kAccCol = 0;
 constexpr int kSfaCol = 256;       // scale-factor column sets start here ...
 constexpr int kSfbCol = 260;       // ... SFA (4 columns) then SFB (8 columns)
 constexpr int kSfSetCols = 12;
-constexpr int kSfSets = 4;         // rotated per k-step so a copy never waits on the MMA
-                                   // still reading the previous k-step's scales
+constexpr int kSfSets = 4;         // rotated (per copy) so that a copy never overwrites the
+                                   // scales an earlier k-step's MMAs may still be reading
 constexpr int kThreads = 256;
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
