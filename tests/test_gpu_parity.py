@@ -289,6 +289,32 @@ def test_small_tiles_equal_single(name):
     assert torch.equal(y1, y2)
 
 
+@pytest.mark.parametrize("wl", [
+    synth.WORKLOADS["v3_fp8"].scaled(T=3000, H=512, E=16, k=4, I=256),
+    synth.WORKLOADS["mixtral_bf16"].scaled(T=2500, H=384, E=5, I=256),
+    synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=2400, H=768, E=64, k=16, I=256),
+], ids=["v3_fp8", "mixtral_bf16_h384", "skewed_fp8_fp4"])
+def test_forward_many_tokens_equals_unfused_chain(wl):
+    """Enough tokens for the persistent kernel's bulk-copy combine (whole 256-column items
+    and a 128-column tail): still the chain's bytes."""
+    d = _inputs(wl)
+    W = weights_of(wl, d)
+    M.moe_set_gemm_tiles("single")
+    try:
+        out = M.moe_forward(d["x"], d["logits"], W, wl.k, wl.score, bias=d["bias"],
+                            x_scales=d["x_scales"])
+        idx, w = M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"])
+        r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
+        y = M.moe_fused_ffn(r["x_perm"], r["expert_offsets"], W,
+                            x_perm_scales=r["x_perm_scales"])
+        out2 = M.moe_combine(y, r["slot_of"], w)
+        torch.cuda.synchronize()
+        assert M.moe_get_device_error()[0] == 0
+    finally:
+        M.moe_set_gemm_tiles("auto")
+    assert torch.equal(out, out2)
+
+
 def test_forward_deterministic():
     wl = SMALL["skewed_fp8_fp4"]
     d = _inputs(wl)
