@@ -32,6 +32,9 @@ takes one plain reading, stated in the function that implements it:
   output are BF16 (fp32 for the fp32 layer); the combine sums the k expert outputs in rank
   order.
 
+``oracle.backward`` (imported by name, not re-exported here) holds the gradients of the
+same layer's fp64 definition, pinned by finite differences and torch autograd.
+
 Every function accumulates in fp64 and applies each storage rounding of the layer's data
 contract at the point where the CUDA path stores that tensor.
 """
