@@ -26,6 +26,11 @@
  *                 power-of-two scale per 128x128 block
  *       MOE_E2M1  OCP MX FP4 codes, two per byte (element 2i in the low nibble), weights
  *                 only, one UE8M0 scale byte (value 2^(b-127)) per 1x32 block along K
+ *     An fp32 scale must be a positive normal power of two (2^-126 .. 2^127): the tensor
+ *     cores take it as a UE8M0 exponent byte.  A GEMM that reads any other scale value
+ *     records MOE_ERR_UNSUPPORTED with site 301 in the device error word and its output
+ *     is undefined (scale values live on the device, so this cannot be checked before the
+ *     launch).
  *   - Supported (activation, weight) pairs: (F32, F32), (BF16, BF16), (E4M3, E4M3),
  *     (E4M3, E2M1).  h (the SwiGLU output) is stored in the activation format (E4M3 with a
  *     power-of-two scale per 1x128 block); y and out are BF16, except F32 for the F32 layer.
@@ -238,9 +243,11 @@ moe_status moe_dispatch_noalloc(const void* x, const float* x_scales, int act, i
 size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, int wt);
 
 /* Synchronises `stream`, then reads and clears the calling device's error word.
- * Returns MOE_OK, or the recorded MOE_ERR_TIMEOUT / MOE_ERR_DEVICE with *site (may be NULL)
- * set to the code location that recorded it, or MOE_ERR_CUDA if the synchronisation
- * itself failed. */
+ * Returns MOE_OK, or the first recorded failure with *site (may be NULL) set to the code
+ * location that recorded it, or MOE_ERR_CUDA if the synchronisation itself failed.
+ * Recorded failures: MOE_ERR_TIMEOUT at a bounded wait (sites 101-106: GEMM pipeline
+ * barriers; 201: the persistent kernel's grid barrier), MOE_ERR_UNSUPPORTED at site 301
+ * (an fp32 block scale that is not a positive normal power of two). */
 moe_status moe_get_device_error(cudaStream_t stream, int* site);
 
 /* Static string naming a status code. */

@@ -24,6 +24,7 @@ enum Site : int {
   SITE_GEMM_SF_EMPTY = 105,  // scale-factor loader waiting for a free smem stage
   SITE_GEMM_DRAIN = 106,     // loader draining its in-flight copies after an abort
   SITE_GRID_BARRIER = 201,   // persistent kernel waiting at a grid-wide barrier
+  SITE_SCALE_FORMAT = 301,   // an fp32 block scale that is not a positive normal power of two
 };
 
 __device__ __forceinline__ void report_error(int* err, int code, int site) {
@@ -386,6 +387,14 @@ __device__ __forceinline__ void tmem_ld_wait() {
 // UE8M0 byte of a positive power-of-two fp32 scale (its biased exponent field).
 __device__ __forceinline__ uint32_t ue8m0_of_pow2(float s) {
   return (__float_as_uint(s) >> 23) & 0xFFu;
+}
+
+// Nonzero when the fp32 bit pattern w is not a positive normal power of two (sign or
+// mantissa bits set, zero / subnormal or Inf / NaN exponent field): such a scale has no
+// exact UE8M0 byte.
+__device__ __forceinline__ uint32_t not_pow2_scale(uint32_t w) {
+  const uint32_t e = (w >> 23) & 0xFFu;
+  return (w & 0x807FFFFFu) | static_cast<uint32_t>(e == 0u || e == 0xFFu);
 }
 
 // Smallest n with a <= 448 * 2^n for a > 0 finite (448 = 1.75 * 2^8).  With

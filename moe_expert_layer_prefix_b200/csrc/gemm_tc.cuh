@@ -586,7 +586,8 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     // atom order (b = sub-block).  kSfBatch slots are published at a time with one warp-wide
     // arrive on the (pair leader's) slot barriers, so the cluster-scope release that makes
     // them visible is paid once per batch; kSfBatch + 4 <= kSfSlots keeps the loader free to
-    // stage every slot a published group needs.
+    // stage every slot a published group needs.  A scale word that is not a positive normal
+    // power of two (no exact UE8M0 byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
     static_assert(kSfBatch + 4 <= kSfSlots, "scale ring too shallow for batch + group");
     if constexpr (kBlockScaled) {
       const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
@@ -594,6 +595,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       const uint32_t it0 = pipe.sf_it;
       const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
       bool ok = true;
+      uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
       for (int b = 0; b < n_iter && ok; b += kSfBatch) {
         const int cnt = n_iter - b < kSfBatch ? n_iter - b : kSfBatch;
         for (int j = 0; j < cnt; ++j) {
@@ -621,10 +623,13 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
               wa1 |= ((a.y >> 23) & 0xFFu) << (8 * q);
               wa2 |= ((a.z >> 23) & 0xFFu) << (8 * q);
               wa3 |= ((a.w >> 23) & 0xFFu) << (8 * q);
+              bad |= not_pow2_scale(a.x) | not_pow2_scale(a.y) | not_pow2_scale(a.z) |
+                     not_pow2_scale(a.w);
               if constexpr (kBFmt != 5) {
                 const uint2 w2 = *reinterpret_cast<const uint2*>(src + kSfaBytes + 16 * lane);
                 wb0 |= ((w2.x >> 23) & 0xFFu) << (8 * q);
                 wb1 |= ((w2.y >> 23) & 0xFFu) << (8 * q);
+                bad |= not_pow2_scale(w2.x) | not_pow2_scale(w2.y);
               }
             }
             uint8_t* dst =
@@ -647,6 +652,8 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
         }
       }
       pipe.sf_it = it0 + n_iter;
+      // the exponent fields were used all the same: the result is undefined, the call fails
+      if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
