@@ -38,7 +38,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # smaller case with the same rows per expert (dram__bytes_read.sum + dram__bytes_write.sum
 # of one launch).  Used for the roofline's "traffic".
 TRAFFIC_RATIO = {
-    ("v3_fp8", "linear1"): (1.154, "the V3-shaped layer at T=1024, E=32"),
+    ("v3_fp8", "linear1"): (1.151, "the V3-shaped layer at T=1024, E=32"),
 }
 
 
