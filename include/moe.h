@@ -17,7 +17,8 @@
  *     gave up) is recorded in a per-device error word read by moe_get_device_error().
  *   - Shapes: T tokens, H hidden, E experts, k experts per token, I expert intermediate
  *     size, S = T*k dispatch slots.  Preconditions: T >= 1, 1 <= k <= min(E, 32),
- *     E <= 1024, H % 128 == 0, I % 128 == 0.
+ *     E <= 1024, H % 128 == 0, I % 128 == 0, S <= 2^31 - 1 (slot indices are 32-bit; a
+ *     larger S returns MOE_ERR_UNSUPPORTED and sizes its workspace to 0).
  *   - Tensor formats (moe_dtype):
  *       MOE_F32   IEEE binary32
  *       MOE_BF16  bfloat16

@@ -1,6 +1,7 @@
 // C ABI of libmoe.so: argument checking, workspace carving and launch sequencing.
 // Every computation happens in the kernels of the other translation units.
 #include <atomic>
+#include <climits>
 #include <mutex>
 
 #include "common.cuh"
@@ -77,10 +78,13 @@ inline bool valid_pair(int act, int wt) {
 
 inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
 
+// Slot indices t*k + j are 32-bit on the device.
+inline bool slots_fit(int T, int k) { return static_cast<long long>(T) * k <= INT32_MAX; }
+
 moe_status check_shapes(int T, int H, int E, int k) {
   if (T < 1 || H < 128 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
   if (H % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  if (E > 1024 || k > 32 || k > E) return MOE_ERR_UNSUPPORTED;
+  if (E > 1024 || k > 32 || k > E || !slots_fit(T, k)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -140,7 +144,7 @@ moe_status moe_set_gemm_tiles(int mode) {
 }
 
 size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, int wt) {
-  if (T < 1 || H < 1 || E < 1 || k < 1 || I < 1) return 0;
+  if (T < 1 || H < 1 || E < 1 || k < 1 || I < 1 || !slots_fit(T, k)) return 0;
   if (!valid_pair(act, wt)) return 0;
   const int S = T * k;
   switch (op) {
@@ -208,7 +212,7 @@ moe_status moe_route_ex(const float* logits, const float* bias, int T, int E, in
   if (logits == nullptr || topk_idx == nullptr || topk_w == nullptr) return MOE_ERR_INVALID_ARG;
   if (T < 1 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
   if (score != MOE_SCORE_SOFTMAX && score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
-  if (E > 1024 || k > 32 || k > E) return MOE_ERR_UNSUPPORTED;
+  if (E > 1024 || k > 32 || k > E || !slots_fit(T, k)) return MOE_ERR_UNSUPPORTED;
   if (!aligned(logits, 4) || !aligned(topk_idx, 4) || !aligned(topk_w, 4) ||
       (bias && !aligned(bias, 4)))
     return MOE_ERR_MISALIGNED;
@@ -320,7 +324,7 @@ moe_status moe_combine(const void* y, int y_dt, const int32_t* slot_of, const fl
                        int T, int k, int H, void* out, int out_dt, cudaStream_t stream) {
   if (!y || !slot_of || !topk_w || !out) return MOE_ERR_INVALID_ARG;
   if (T < 1 || k < 1 || H < 8) return MOE_ERR_INVALID_ARG;
-  if (k > 32 || H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (k > 32 || H % 8 != 0 || !slots_fit(T, k)) return MOE_ERR_UNSUPPORTED;
   if ((y_dt != MOE_F32 && y_dt != MOE_BF16) || (out_dt != MOE_F32 && out_dt != MOE_BF16))
     return MOE_ERR_INVALID_ARG;
   if (!aligned(y, 16) || !aligned(out, 16) || !aligned(slot_of, 4) || !aligned(topk_w, 4))

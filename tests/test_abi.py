@@ -79,3 +79,19 @@ def test_argument_errors_need_no_gpu():
     g = M.MoeRouterGroups(3, 1, 1.0)                                  # 256 experts / 3 groups
     st = M._route_ex(fake, None, 4, 256, 8, 0, 1, ctypes.byref(g), fake, fake, None)
     assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
+
+
+def test_slot_count_beyond_32_bits_is_refused_before_launch():
+    # slot indices t*k + j are 32-bit on the device: T*k > 2^31 - 1 is refused, and sizes
+    # to zero, on the host (the dummy addresses are never dereferenced)
+    import ctypes
+    fake = ctypes.c_void_p(1 << 20)
+    T = (1 << 31) // 8                                                 # T * 8 = 2^31
+    st = M._route_ex(fake, None, T, 256, 8, 0, 1, None, fake, fake, None)
+    assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
+    st = M._dispatch_quant(fake, T, 256, 256, 8, fake, fake, fake, fake, fake, fake, fake,
+                           1 << 40, None)
+    assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
+    assert M.moe_workspace_size("forward", T, 7168, 256, 8, 2048, "e4m3", "e4m3") == 0
+    assert M.moe_workspace_size("forward", T - 1, 7168, 256, 8, 2048, "e4m3", "e4m3") > 0
+
