@@ -295,8 +295,8 @@ def test_small_tiles_equal_single(name):
     synth.WORKLOADS["skewed_fp8_fp4"].scaled(T=2400, H=768, E=64, k=16, I=256),
 ], ids=["v3_fp8", "mixtral_bf16_h384", "skewed_fp8_fp4"])
 def test_forward_many_tokens_equals_unfused_chain(wl):
-    """Enough tokens for the persistent kernel's bulk-copy combine (whole 256-column items
-    and a 128-column tail): still the chain's bytes."""
+    """Enough tokens (T >= 2 x the persistent kernel's warps) for its whole-row combine
+    path: still the chain's bytes."""
     d = _inputs(wl)
     W = weights_of(wl, d)
     M.moe_set_gemm_tiles("single")
