@@ -202,3 +202,64 @@ def layer_backward(L: Layer, dout, n_group: int = 1, topk_group: int = 0, scale:
     w1, w2 = _weights_f64(L)
     return backward_values(L.x_hat(), L.logits, L.bias, w1, w2, L.k, L.score, dout, L.renorm,
                            n_group, topk_group, scale)
+
+
+def layer_backward_stored(L: Layer, dout, store=None):
+    """The backward of a BF16 layer with every intermediate stored where the CUDA path stores
+    it (`store` rounds a value to its storage format; default BF16 round-to-nearest-even):
+
+      forward tensors, as the forward pass stores them:
+        h = store(silu(g) * u),  y = store(h W2^T),  gates w as fp32
+      dgates[t, j] = dout[t] . y[slot(t, j)]         (an fp32 result: kept exact here)
+      dy_w[slot]   = store(w[t, j] * dout[t])
+      G            = store(x W1^T)                    (pre-activations, recomputed)
+      dh           = store(dy_w W2)
+      dG           = store(swiglu_grad(G, dh))        (gate and up halves)
+      dx_slot      = store(dG W1),   dx[t] = store(sum over the token's slots of dx_slot)
+      dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e        (fp32 results: exact here)
+      dlogits      = gate_grad(dgates)                (an fp32 result)
+
+    With store = identity this is layer_backward up to the fp32 storage of the gates.
+    Returns the same dict as layer_backward."""
+    from .formats import round_bf16
+    st = round_bf16 if store is None else store
+    dout = np.asarray(dout, np.float64)
+    idx, w = route(L.logits, L.bias, L.k, L.score, L.renorm)
+    w32 = w.astype(np.float32).astype(np.float64)
+    _, offsets, perm_src, _ = dispatch(idx, L.E)
+    tok = perm_src // L.k
+    rank = perm_src % L.k
+    xh = L.x_hat()
+    T, H = xh.shape
+    dx_slot = np.zeros((tok.size, H), np.float64)
+    dgates = np.zeros_like(w)
+    dw1 = dw2 = None
+    for e in range(L.E):
+        a, b = int(offsets[e]), int(offsets[e + 1])
+        w1, w2 = L.expert_weights(e)
+        if dw1 is None:
+            dw1 = np.zeros((L.E,) + w1.shape, np.float64)
+            dw2 = np.zeros((L.E,) + w2.shape, np.float64)
+        if a == b:
+            continue
+        I = w1.shape[0] // 2
+        t, j = tok[a:b], rank[a:b]
+        x = xh[t]
+        _, gate, up, _ = expert_ffn_exact(x, w1, w2)
+        h = st(gate * _sigmoid(gate) * up)
+        y = st(h @ w2.T)
+        dgates[t, j] = np.einsum("nh,nh->n", dout[t], y)
+        dyw = st(w32[t, j][:, None] * dout[t])
+        G = st(x @ w1.T)
+        dh = st(dyw @ w2)
+        dg, du = swiglu_grad(G[:, :I], G[:, I:], dh)
+        dG = np.concatenate([st(dg), st(du)], axis=1)
+        dx_slot[a:b] = st(dG @ w1)
+        dw1[e] = dG.T @ x
+        dw2[e] = dyw.T @ h
+    dx = np.zeros((T, H), np.float64)
+    np.add.at(dx, tok, dx_slot)
+    dl = gate_grad(L.logits, idx, dgates, L.score, L.renorm)
+    dbias = None if L.bias is None else np.zeros(L.E, np.float64)
+    return dict(dx=st(dx), dw1=dw1, dw2=dw2, dlogits=dl, dbias=dbias, topk_idx=idx,
+                offsets=offsets)

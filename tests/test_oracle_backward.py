@@ -178,3 +178,37 @@ def test_forward_exact_is_the_oracle_forward_before_rounding():
     assert np.max(np.abs(a - b)) <= 1e-6 * np.sqrt(np.mean(b * b))
     g = B.layer_backward(L, rng.standard_normal((T, H)))
     assert g["dx"].shape == (T, H) and g["dw1"].shape == (E, 2 * I, H)
+
+
+def _bf16_layer(seed, score="softmax", renorm=True, bias=False, T=40, H=256, E=6, k=2, I=128):
+    import synth
+    from tests.util import oracle_layer
+    wl = synth.WORKLOADS["mixtral_bf16"].scaled(T=T, H=H, E=E, k=k, I=I, score=score,
+                                                bias=bias, renorm=renorm)
+    d = synth.make_inputs(wl, "cpu")
+    L = oracle_layer(wl, d)
+    dout = oracle.round_bf16(np.random.default_rng(seed).standard_normal((T, H)))
+    return L, dout
+
+
+@pytest.mark.parametrize("score,renorm,bias", [("softmax", True, False),
+                                               ("softmax", False, False),
+                                               ("sigmoid", True, True)])
+def test_stored_backward_without_rounding_is_the_exact_backward(score, renorm, bias):
+    L, dout = _bf16_layer(4, score, renorm, bias)
+    a = B.layer_backward_stored(L, dout, store=lambda v: v)
+    b = B.layer_backward(L, dout)
+    assert np.array_equal(a["topk_idx"], b["topk_idx"])
+    for n in ("dx", "dw1", "dw2", "dlogits"):
+        # the only difference: the gates stored as fp32
+        assert np.allclose(a[n], b[n], rtol=1e-6, atol=1e-6 * np.abs(b[n]).max()), n
+
+
+def test_stored_backward_is_close_to_the_exact_backward():
+    """BF16 storage of the intermediates moves every gradient by well under 1 % (rel-L2)."""
+    L, dout = _bf16_layer(5)
+    a = B.layer_backward_stored(L, dout)
+    b = B.layer_backward(L, dout)
+    for n in ("dx", "dw1", "dw2", "dlogits"):
+        rel = np.sqrt(np.sum((a[n] - b[n]) ** 2) / np.sum(b[n] ** 2))
+        assert 0 < rel < 1e-2, (n, rel)
