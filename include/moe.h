@@ -68,7 +68,8 @@ typedef enum moe_op {
   MOE_OP_LINEAR1 = 2,
   MOE_OP_LINEAR2 = 3,
   MOE_OP_FUSED_FFN = 4,
-  MOE_OP_FORWARD = 5
+  MOE_OP_FORWARD = 5,
+  MOE_OP_BACKWARD = 6
 } moe_op;
 
 /* Expert weights.  W1 [E, 2I, H]: rows [0, I) are the gate projection, rows [I, 2I) the up
@@ -219,6 +220,61 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
                           const moe_weights* W, void* out, int32_t* topk_idx, float* topk_w,
                           int32_t* expert_offsets, void* ws, size_t ws_bytes,
                           cudaStream_t stream);
+
+/* Batched transpose: dst[e] = src[e]^T for src [E, R, C] row-major, dst [E, C, R].
+ * (youleyou, section "Tile Kernels：逼近硬件极限的底层优化", feature list, batched matrix
+ *  transpose item.)  Makes the transposed weight copies the backward's GEMMs read
+ * (W1^T [E, H, 2I], W2^T [E, I, H]).
+ *   dtype  element size: MOE_F32 (4 bytes), MOE_BF16 (2), MOE_E4M3 (1); E2M1 (packed
+ *          nibbles) returns MOE_ERR_UNSUPPORTED.
+ *   src, dst device buffers of E*R*C elements; they must not overlap. */
+moe_status moe_transpose_experts(const void* src, int dtype, int E, int R, int C, void* dst,
+                                 cudaStream_t stream);
+
+/* Inputs and outputs of moe_expert_backward (all device pointers; S = T*k). */
+typedef struct moe_backward_args {
+  int T, H, E, k, I;
+  int score;        /* moe_score of the forward router */
+  int renorm;       /* the forward's renorm flag */
+  float scale;      /* the forward's routed scaling factor (1 for moe_forward) */
+  const void* dout; /* BF16 [T, H]: gradient of the layer output */
+  const float* logits;           /* fp32 [T, E], as given to the forward */
+  const int32_t* topk_idx;       /* int32 [T, k], the forward's selection */
+  const float* topk_w;           /* fp32 [T, k], the forward's gates */
+  const int32_t* expert_offsets; /* int32 [E+1]  (moe_dispatch) */
+  const int32_t* slot_of;        /* int32 [T*k]  (moe_dispatch) */
+  const void* x_perm;            /* BF16 [S, H]  (moe_dispatch) */
+  const void* h;                 /* BF16 [S, I]  (moe_expert_linear1) */
+  const void* y;                 /* BF16 [S, H]  (moe_expert_linear2) */
+  const void* w1;                /* BF16 [E, 2I, H] */
+  const void* w2;                /* BF16 [E, H, I] (read through w2_t only) */
+  const void* w1_t;              /* BF16 [E, H, 2I] = W1^T (moe_transpose_experts) */
+  const void* w2_t;              /* BF16 [E, I, H]  = W2^T (moe_transpose_experts) */
+  void* dx;                      /* out BF16 [T, H] */
+  float* dw1;                    /* out fp32 [E, 2I, H]; experts no token picked get 0 */
+  float* dw2;                    /* out fp32 [E, H, I] */
+  float* dlogits;                /* out fp32 [T, E] */
+} moe_backward_args;
+
+/* Backward of the BF16 layer: the gradients of out = sum_j w[t, j] * W2_e SwiGLU(W1_e x_t)
+ * with respect to x, W1, W2 and the router logits, the top-k selection held fixed (it is
+ * piecewise constant; the sigmoid router's selection bias gets no gradient).
+ * (youleyou, section "Tile Kernels：逼近硬件极限的底层优化", feature list, model-layer item:
+ *  wrappers that make the kernels trainable layers.)
+ * Steps, each stored where the comment says:
+ *   combine backward:  dy_w[slot] = BF16(w * dout[t]);  dgate = dout[t] . y[slot] (fp32)
+ *   router backward:   dlogits (fp32) through the gate function
+ *   G  = BF16(x_perm W1^T)  (pre-activations recomputed on the expert GEMM)
+ *   dh = BF16(dy_w W2)       (expert GEMM on W2^T)
+ *   dG = BF16(SwiGLU backward of G, dh)
+ *   dx_slot = BF16(dG W1)    (expert GEMM on W1^T);  dx[t] = BF16(sum of its k slots)
+ *   dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e  (fp32)
+ * BF16 layers only (the arguments carry no formats).  BF16 tensors, dw1 and dw2 must be
+ * 16-byte aligned, the other arrays 4-byte aligned.  Workspace:
+ * moe_workspace_size(MOE_OP_BACKWARD, T, H, E, k, I, MOE_BF16, MOE_BF16) bytes, 256-byte
+ * aligned.  Deterministic: no atomics; every sum runs in a fixed order. */
+moe_status moe_expert_backward(const moe_backward_args* args, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
 
 /* moe_dispatch without a caller workspace, for callers that cannot allocate device memory
  * (a host with no device allocator of its own, a runtime that forbids allocations after

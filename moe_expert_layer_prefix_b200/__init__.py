@@ -29,19 +29,27 @@ STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED",
           -6: "MOE_ERR_TIMEOUT", -7: "MOE_ERR_DEVICE"}
 DTYPES = {"f32": 0, "bf16": 1, "e4m3": 2, "e2m1": 3}
 SCORES = {"softmax": 0, "sigmoid": 1}
-OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5}
+OPS = {"dispatch": 1, "linear1": 2, "linear2": 3, "fused_ffn": 4, "forward": 5, "backward": 6}
 
 EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear2",
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
            "moe_get_device_error", "moe_status_string", "moe_launch_count",
            "moe_dispatch_noalloc", "moe_set_gemm_tiles", "moe_dispatch_quant", "moe_route_ex",
-           "moe_forward_ex")
+           "moe_forward_ex", "moe_transpose_experts", "moe_expert_backward")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
 
 class MoeRouterGroups(ctypes.Structure):
     _fields_ = [("n_group", ctypes.c_int), ("topk_group", ctypes.c_int), ("scale", ctypes.c_float)]
+
+
+class MoeBackwardArgs(ctypes.Structure):
+    _fields_ = ([(n, ctypes.c_int) for n in ("T", "H", "E", "k", "I", "score", "renorm")] +
+                [("scale", ctypes.c_float)] +
+                [(n, _P) for n in ("dout", "logits", "topk_idx", "topk_w", "expert_offsets",
+                                   "slot_of", "x_perm", "h", "y", "w1", "w2", "w1_t", "w2_t",
+                                   "dx", "dw1", "dw2", "dlogits")])
 
 
 class MoeWeights(ctypes.Structure):
@@ -76,6 +84,8 @@ _forward = _sig("moe_forward", _I, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
 _forward_ex = _sig("moe_forward_ex", _I, [_P, _P, _P, _P, _I, _I, ctypes.POINTER(MoeRouterGroups),
                                           _I, _I, _I, _I, _I, ctypes.POINTER(MoeWeights), _P, _P,
                                           _P, _P, _P, _Z, _P])
+_transpose = _sig("moe_transpose_experts", _I, [_P, _I, _I, _I, _I, _P, _P])
+_backward = _sig("moe_expert_backward", _I, [ctypes.POINTER(MoeBackwardArgs), _P, _Z, _P])
 _ws_size = _sig("moe_workspace_size", _Z, [_I, _I, _I, _I, _I, _I, _I, _I])
 _get_err = _sig("moe_get_device_error", _I, [_P, ctypes.POINTER(ctypes.c_int)])
 _status_string = _sig("moe_status_string", ctypes.c_char_p, [_I])
@@ -330,3 +340,43 @@ def moe_dispatch_noalloc(x, topk_idx, E, act, out, x_scales=None, stream=None):
                              _ptr(out["expert_offsets"]), _ptr(out["perm_src"]),
                              _ptr(out["slot_of"]), _stream(stream)), "moe_dispatch_noalloc")
     return out
+
+
+_ELEM_DTYPE = {torch.float32: "f32", torch.bfloat16: "bf16", torch.uint8: "e4m3"}
+
+
+def moe_transpose_experts(src, out=None, stream=None):
+    """dst[e] = src[e]^T for a [E, R, C] tensor (fp32, BF16 or one-byte codes)."""
+    E, R, C = src.shape
+    if out is None:
+        out = torch.empty((E, C, R), dtype=src.dtype, device=src.device)
+    _check(_transpose(_ptr(src), DTYPES[_ELEM_DTYPE[src.dtype]], E, R, C, _ptr(out),
+                      _stream(stream)), "moe_transpose_experts")
+    return out
+
+
+def moe_expert_backward(dout, logits, topk_idx, topk_w, expert_offsets, slot_of, x_perm, h, y,
+                        W: Weights, w1_t, w2_t, k, score="softmax", renorm=True, scale=1.0,
+                        ws=None, stream=None):
+    """Backward of the BF16 layer from the forward's tensors (see include/moe.h); w1_t, w2_t
+    are moe_transpose_experts of W.w1, W.w2.  Returns dict(dx, dw1, dw2, dlogits)."""
+    T, H = dout.shape
+    E = logits.shape[1]
+    I = h.shape[1]
+    dev = dout.device
+    g = dict(dx=torch.empty((T, H), dtype=torch.bfloat16, device=dev),
+             dw1=torch.empty((E, 2 * I, H), dtype=torch.float32, device=dev),
+             dw2=torch.empty((E, H, I), dtype=torch.float32, device=dev),
+             dlogits=torch.empty((T, E), dtype=torch.float32, device=dev))
+    a = MoeBackwardArgs(T, H, E, k, I, SCORES[score], int(bool(renorm)), float(scale),
+                        _ptr(dout), _ptr(logits), _ptr(topk_idx), _ptr(topk_w),
+                        _ptr(expert_offsets), _ptr(slot_of), _ptr(x_perm), _ptr(h), _ptr(y),
+                        _ptr(W.w1), _ptr(W.w2), _ptr(w1_t), _ptr(w2_t), _ptr(g["dx"]),
+                        _ptr(g["dw1"]), _ptr(g["dw2"]), _ptr(g["dlogits"]))
+    need = moe_workspace_size("backward", T, H, E, k, I, "bf16", "bf16")
+    if ws is None:
+        ws = workspace(need, dev)
+    _check(_backward(ctypes.byref(a), _ptr(ws), ws.numel(), _stream(stream)),
+           "moe_expert_backward")
+    return g
+

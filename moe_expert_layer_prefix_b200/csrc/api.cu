@@ -155,6 +155,15 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       return 0;
     case MOE_OP_FUSED_FFN:
       return h_bytes(S, I, act);
+    case MOE_OP_BACKWARD: {
+      if (act != MOE_BF16 || wt != MOE_BF16) return 0;
+      size_t b = 0;
+      b += round256(static_cast<size_t>(S) * H * 2) * 2;      // dy_w, dx_slot
+      b += round256(static_cast<size_t>(S) * 2 * I * 2) * 2;  // G, dG
+      b += round256(static_cast<size_t>(S) * I * 2);          // dh
+      b += round256(static_cast<size_t>(S) * 4) * 2;          // dgates, unit weights
+      return b;
+    }
     case MOE_OP_FORWARD: {
       size_t b = 0;
       b += round256(static_cast<size_t>(S) * 4);                       // topk_idx
@@ -443,6 +452,99 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
   if (st != MOE_OK) return st;
   const int ydt = act == MOE_F32 ? MOE_F32 : MOE_BF16;
   return moe_combine(y, ydt, slot_of, topk_w, T, k, H, out, ydt, stream);
+}
+
+moe_status moe_transpose_experts(const void* src, int dtype, int E, int R, int C, void* dst,
+                                 cudaStream_t stream) {
+  if (!src || !dst || E < 1 || R < 1 || C < 1) return MOE_ERR_INVALID_ARG;
+  int eb = 0;
+  switch (dtype) {
+    case MOE_F32: eb = 4; break;
+    case MOE_BF16: eb = 2; break;
+    case MOE_E4M3: eb = 1; break;
+    case MOE_E2M1: return MOE_ERR_UNSUPPORTED;
+    default: return MOE_ERR_INVALID_ARG;
+  }
+  if (E > 65535 || (R + 31) / 32 > 65535) return MOE_ERR_UNSUPPORTED;  // grid limits
+  if (!aligned(src, eb) || !aligned(dst, eb)) return MOE_ERR_MISALIGNED;
+  const uintptr_t n = static_cast<uintptr_t>(E) * R * C * eb;
+  const uintptr_t s0 = reinterpret_cast<uintptr_t>(src), d0 = reinterpret_cast<uintptr_t>(dst);
+  if (s0 < d0 + n && d0 < s0 + n) return MOE_ERR_INVALID_ARG;  // overlapping buffers
+  return cuda_status(launch_transpose(src, eb, E, R, C, dst, stream));
+}
+
+moe_status moe_expert_backward(const moe_backward_args* a, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+  if (a == nullptr) return MOE_ERR_INVALID_ARG;
+  moe_status st = check_shapes(a->T, a->H, a->E, a->k);
+  if (st != MOE_OK) return st;
+  if (a->I < 128) return MOE_ERR_INVALID_ARG;
+  if (a->I % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (a->score != MOE_SCORE_SOFTMAX && a->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (!(a->scale == a->scale) || a->scale == INFINITY || a->scale == -INFINITY)
+    return MOE_ERR_INVALID_ARG;
+  const void* bf[] = {a->dout, a->x_perm, a->h, a->y, a->w1, a->w1_t, a->w2_t, a->dx,
+                      a->dw1, a->dw2};
+  for (const void* q : bf) {
+    if (q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned(q, 16)) return MOE_ERR_MISALIGNED;
+  }
+  const void* w4[] = {a->logits, a->topk_idx, a->topk_w, a->expert_offsets, a->slot_of,
+                      a->dlogits};
+  for (const void* q : w4) {
+    if (q == nullptr) return MOE_ERR_INVALID_ARG;
+    if (!aligned(q, 4)) return MOE_ERR_MISALIGNED;
+  }
+  const int T = a->T, H = a->H, E = a->E, k = a->k, I = a->I, S = T * k;
+  const size_t need = moe_workspace_size(MOE_OP_BACKWARD, T, H, E, k, I, MOE_BF16, MOE_BF16);
+  if (!ws || !aligned(ws, 256) || ws_bytes < need) return MOE_ERR_WORKSPACE;
+  char* p = static_cast<char*>(ws);
+  auto take = [&p](size_t bytes) {
+    void* q = p;
+    p += round256(bytes);
+    return q;
+  };
+  void* dy_w = take(static_cast<size_t>(S) * H * 2);
+  void* dx_slot = take(static_cast<size_t>(S) * H * 2);
+  void* G = take(static_cast<size_t>(S) * 2 * I * 2);
+  void* dG = take(static_cast<size_t>(S) * 2 * I * 2);
+  void* dh = take(static_cast<size_t>(S) * I * 2);
+  float* dgates = static_cast<float*>(take(static_cast<size_t>(S) * 4));
+  float* ones = static_cast<float*>(take(static_cast<size_t>(S) * 4));
+  int* err = device_error_word();
+  // combine and router backward
+  if (launch_combine_backward(a->dout, a->y, a->slot_of, a->topk_w, T, k, H, dy_w, dgates,
+                              stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_gate_backward(a->logits, a->topk_idx, dgates, T, E, k,
+                           a->score == MOE_SCORE_SIGMOID, a->renorm != 0, a->scale, a->dlogits,
+                           stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  // expert GEMM of the forward pass, out[S, N] = A[S, K] . W[E, N, K]^T: FfnArgs with
+  // I = K and H = N (its linear-2 form)
+  const FfnArgs g_args{MOE_BF16, MOE_BF16, a->x_perm, nullptr, a->expert_offsets, S, 2 * I, H,
+                       E, a->w1, nullptr, G, nullptr, err};
+  if (launch_linear2_tc(g_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const FfnArgs dh_args{MOE_BF16, MOE_BF16, dy_w, nullptr, a->expert_offsets, S, I, H,
+                        E, a->w2_t, nullptr, dh, nullptr, err};
+  if (launch_linear2_tc(dh_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  if (launch_swiglu_backward(G, dh, S, I, dG, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  const FfnArgs dx_args{MOE_BF16, MOE_BF16, dG, nullptr, a->expert_offsets, S, H, 2 * I,
+                        E, a->w1_t, nullptr, dx_slot, nullptr, err};
+  if (launch_linear2_tc(dx_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  // dx[t] = sum of the token's slot rows (the combine with unit weights)
+  if (launch_fill(ones, static_cast<size_t>(S), 1.0f, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_combine(dx_slot, 0, a->slot_of, ones, T, k, H, a->dx, 0, stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  // weight gradients
+  if (launch_wgrad(dG, a->x_perm, a->expert_offsets, E, 2 * I, H, a->dw1, stream) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (launch_wgrad(dy_w, a->h, a->expert_offsets, E, H, I, a->dw2, stream) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 }  // extern "C"

@@ -32,6 +32,21 @@ cudaError_t launch_dispatch(const void* x, const float* x_scales, int row_bytes,
 cudaError_t launch_combine(const void* y, int y_f32, const int32_t* slot_of, const float* topk_w,
                            int T, int k, int H, void* out, int out_f32, cudaStream_t s);
 
+// Backward (BF16 layer) steps other than the expert GEMMs (backward.cu).
+cudaError_t launch_transpose(const void* src, int elem_bytes, int E, int R, int C, void* dst,
+                             cudaStream_t s);
+cudaError_t launch_combine_backward(const void* dout, const void* y, const int32_t* slot_of,
+                                    const float* topk_w, int T, int k, int H, void* dy_w,
+                                    float* dgates, cudaStream_t s);
+cudaError_t launch_gate_backward(const float* logits, const int32_t* topk_idx,
+                                 const float* dgates, int T, int E, int k, int sigmoid,
+                                 int renorm, float scale, float* dlogits, cudaStream_t s);
+cudaError_t launch_swiglu_backward(const void* G, const void* dh, int S, int I, void* dG,
+                                   cudaStream_t s);
+cudaError_t launch_wgrad(const void* A, const void* B, const int32_t* offsets, int E, int M,
+                         int N, float* out, cudaStream_t s);
+cudaError_t launch_fill(float* p, size_t n, float v, cudaStream_t s);
+
 struct FfnArgs {
   int act, wt;                 // moe_dtype
   const void* a;               // x_perm (linear-1) or h (linear-2)

@@ -95,3 +95,20 @@ def test_slot_count_beyond_32_bits_is_refused_before_launch():
     assert M.moe_workspace_size("forward", T, 7168, 256, 8, 2048, "e4m3", "e4m3") == 0
     assert M.moe_workspace_size("forward", T - 1, 7168, 256, 8, 2048, "e4m3", "e4m3") > 0
 
+
+
+def test_backward_arguments_are_checked_before_launch():
+    import ctypes
+    fake = ctypes.c_void_p(1 << 20)
+    assert M.moe_status_string(M._backward(None, None, 0, None)) == "MOE_ERR_INVALID_ARG"
+    a = M.MoeBackwardArgs(64, 256, 8, 2, 128, 0, 1, 1.0)     # every pointer NULL
+    assert M.moe_status_string(M._backward(ctypes.byref(a), fake, 1 << 30, None)) == \
+        "MOE_ERR_INVALID_ARG"
+    assert M.moe_workspace_size("backward", 64, 256, 8, 2, 128, "bf16", "bf16") >= \
+        64 * 2 * (256 * 2 * 2 + 256 * 2 * 2 + 128 * 2)
+    assert M.moe_workspace_size("backward", 64, 256, 8, 2, 128, "e4m3", "e4m3") == 0
+    # transposes: packed E2M1 is refused, overlapping buffers too
+    st = M._transpose(fake, M.DTYPES["e2m1"], 2, 64, 64, ctypes.c_void_p(1 << 30), None)
+    assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
+    st = M._transpose(fake, M.DTYPES["bf16"], 2, 64, 64, ctypes.c_void_p((1 << 20) + 64), None)
+    assert M.moe_status_string(st) == "MOE_ERR_INVALID_ARG"
