@@ -260,7 +260,7 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s) {
-  // the dispatch phases keep per-warp masks (8 x E words) in the 64 KB of A stages
+  // the dispatch phases keep per-warp masks (8 x E words) in the idle GEMM ring
   if (a.E > 1024) return cudaErrorNotSupported;
   const bool small = gemm_tile_shape(a.act, a.T * a.k, a.E, false) == 3;
   if (a.act == MOE_BF16 && a.wt == MOE_BF16)
