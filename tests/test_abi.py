@@ -112,3 +112,41 @@ def test_backward_arguments_are_checked_before_launch():
     assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
     st = M._transpose(fake, M.DTYPES["bf16"], 2, 64, 64, ctypes.c_void_p((1 << 20) + 64), None)
     assert M.moe_status_string(st) == "MOE_ERR_INVALID_ARG"
+
+
+def _header_struct(name):
+    """(field, C type) pairs of `typedef struct name {...}` in include/moe.h, in order."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    body = {m.group(2): m.group(1)
+            for m in re.finditer(r"typedef struct(?: \w+)? \{(.*?)\}\s*(\w+);", src, re.S)}[name]
+    body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+    fields = []
+    for decl in body.split(";"):
+        decl = decl.strip()
+        if not decl:
+            continue
+        m = re.match(r"((?:const\s+)?\w+\s*\**)\s*(.*)", decl, re.S)
+        base = m.group(1).replace(" ", "")
+        for part in m.group(2).split(","):
+            part = part.strip()
+            stars = len(part) - len(part.lstrip("*"))
+            fields.append((part.lstrip("*").strip(), "ptr" if "*" in base or stars else base))
+    return fields
+
+
+def _ctypes_kind(t):
+    import ctypes
+    if t is ctypes.c_void_p:
+        return "ptr"
+    return {ctypes.c_int: "int", ctypes.c_float: "float"}[t]
+
+
+def test_binding_structs_match_the_header():
+    # the ctypes mirrors of the header's structs: same fields, same order, same kinds
+    for cname, py in (("moe_weights", M.MoeWeights), ("moe_router_groups", M.MoeRouterGroups),
+                      ("moe_backward_args", M.MoeBackwardArgs)):
+        hdr = _header_struct(cname)
+        mine = [(n, _ctypes_kind(t)) for n, t in py._fields_]
+        assert [n for n, _ in hdr] == [n for n, _ in mine], cname
+        for (n, ht), (_, pk) in zip(hdr, mine):
+            assert (ht == "ptr") == (pk == "ptr") and (ht != "float" or pk == "float"), (cname, n)
