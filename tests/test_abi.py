@@ -150,3 +150,15 @@ def test_binding_structs_match_the_header():
         assert [n for n, _ in hdr] == [n for n, _ in mine], cname
         for (n, ht), (_, pk) in zip(hdr, mine):
             assert (ht == "ptr") == (pk == "ptr") and (ht != "float" or pk == "float"), (cname, n)
+
+
+def test_binding_argument_counts_match_the_header():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    decls = {m.group(1): m.group(2) for m in re.finditer(
+        r"^\s*(?:moe_status|size_t|const char\*|uint64_t)\s+(moe_\w+)\((.*?)\);", src, re.M | re.S)}
+    assert set(decls) == set(M.EXPORTS)
+    for name, params in decls.items():
+        params = params.strip()
+        n = 0 if params in ("", "void") else params.count(",") + 1
+        assert len(getattr(M._lib, name).argtypes or []) == n, name
