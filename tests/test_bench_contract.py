@@ -37,3 +37,29 @@ def test_too_few_warmup_steps_are_rejected():
                timeout=120)
     assert r.returncode != 0
     assert "warmup" in r.stderr
+
+
+def test_algorithmic_units_match_the_published_workload_figures():
+    """The roofline's algorithmic FLOPs and weight bytes against figures computed by hand: the
+    two GEMMs are 6 S H I FLOP (V3 5.772 TFLOP, Mixtral 2.886 TFLOP, decode 90.2 GFLOP); all
+    experts' weights are 11.27 GB for V3 (E4M3 codes + fp32 128x128 scales) and 2.82 GB for
+    Mixtral (BF16)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    for name, tflop in (("v3_fp8", 5.772), ("mixtral_bf16", 2.886), ("decode_fp8_fp4", 0.0902)):
+        wl = synth.WORKLOADS[name]
+        a = bench.algorithmic(wl, wl.E)
+        total = a["linear1"]["flops"] + a["linear2"]["flops"]
+        assert abs(total / 1e12 - tflop) / tflop < 5e-4, (name, total)
+    v3 = synth.WORKLOADS["v3_fp8"]
+    a = bench.algorithmic(v3, v3.E)
+    act = v3.S * (v3.H + v3.H // 128 * 4) + v3.S * (v3.I + v3.I // 128 * 4)
+    weights = a["linear1"]["bytes"] - act + (a["linear2"]["bytes"] - v3.S * (v3.I + v3.I // 128 * 4)
+                                             - v3.S * v3.H * 2)
+    assert abs(weights / 1e9 - 11.27) < 0.01, weights
+    mx = synth.WORKLOADS["mixtral_bf16"]
+    a = bench.algorithmic(mx, mx.E)
+    weights = (a["linear1"]["bytes"] - mx.S * (mx.H + mx.I) * 2 +
+               a["linear2"]["bytes"] - mx.S * mx.I * 2 - mx.S * mx.H * 2)
+    assert abs(weights / 1e9 - 2.82) < 0.01, weights
