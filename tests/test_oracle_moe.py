@@ -362,3 +362,23 @@ def test_route_grouped_excludes_a_strong_expert_in_a_weak_group():
     keys = np.array([[5.0, -9, -9, -9, 3, 3, -9, -9, 2.9, 2.9, -9, -9]], np.float32)
     idx, _ = oracle.route(keys, None, 2, "softmax", n_group=3, topk_group=2)
     assert idx.tolist() == [[4, 5]]
+
+
+def test_dequant_takes_any_fp32_block_scale():
+    """The oracle's dequantisation is code x block scale for any fp32 scale, not only powers of
+    two (the GPU path refuses other scales; the definition does not depend on them)."""
+    rng = np.random.default_rng(12)
+    w = rng.integers(0, 256, (256, 384), dtype=np.uint8)
+    w[(w & 0x7F) == 0x7F] = 0                                  # no NaN codes
+    s = rng.uniform(0.1, 3.0, (2, 3)).astype(np.float32)       # non-power-of-two scales
+    d = oracle.dequant_w(w, s, "e4m3")
+    for _ in range(200):
+        r, c = int(rng.integers(0, 256)), int(rng.integers(0, 384))
+        assert d[r, c] == _bf_dequant_w(w, s, "e4m3", r, c)
+    x = rng.integers(0, 256, (5, 256), dtype=np.uint8)
+    x[(x & 0x7F) == 0x7F] = 0
+    xs = rng.uniform(0.1, 3.0, (5, 2)).astype(np.float32)
+    dx = oracle.dequant_x(x, xs, "e4m3")
+    ref = torch.from_numpy(x).view(torch.float8_e4m3fn).double().numpy() * \
+        np.repeat(xs.astype(np.float64), 128, axis=1)
+    assert np.array_equal(dx, ref)
