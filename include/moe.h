@@ -181,8 +181,16 @@ moe_status moe_expert_linear2(const void* h, const float* h_scales, const int32_
                               int S, int H, int I, int E, const moe_weights* W, void* y, void* ws,
                               size_t ws_bytes, cudaStream_t stream);
 
-/* linear-1 + SwiGLU + linear-2 with h kept in the workspace
- * (moe_workspace_size(MOE_OP_FUSED_FFN, ...) bytes). */
+/* The expert FFN of the dispatched rows: linear-1 + SwiGLU (+ h requantisation for E4M3)
+ * followed by linear-2, y[p] = W2[e] . SwiGLU(W1[e] . x_perm[p]) for every slot p of
+ * expert e, with h kept in the workspace (moe_workspace_size(MOE_OP_FUSED_FFN, ...) bytes,
+ * 256-byte aligned).
+ * (jiqizhixin, section "Mega MoE 是什么？", pipeline paragraph: a linear layer, the SwiGLU
+ *  activation and a second linear layer between dispatch and combine; youleyou, section
+ *  "Tile Kernels：逼近硬件极限的底层优化", feature list, quantisation item: FP8 quantisation
+ *  fused with SwiGLU.)
+ *   Arguments as moe_expert_linear1 / moe_expert_linear2; y [S, H] out.  Errors: those of
+ *   the two calls, and MOE_ERR_WORKSPACE for a missing, misaligned or short workspace. */
 moe_status moe_fused_ffn(const void* x_perm, const float* x_perm_scales,
                          const int32_t* expert_offsets, int S, int H, int I, int E,
                          const moe_weights* W, void* y, void* ws, size_t ws_bytes,
@@ -286,8 +294,9 @@ moe_status moe_expert_backward(const moe_backward_args* args, void* ws, size_t w
  *   loads it until the process exits.  Shapes whose dispatch workspace exceeds it
  *   (moe_workspace_size(MOE_OP_DISPATCH, ...) > 4 MiB; e.g. T > 32736 at E = 1024) return
  *   MOE_ERR_WORKSPACE before anything is launched.
- *   The first call on each device looks up the buffer's device address (with that device
- *   current); make that first call before any stream capture.
+ *   Every call looks up the buffer's device address on the caller's current device (no
+ *   address is cached).  The first call on a device also loads the library's module there;
+ *   make that first call before any stream capture.
  *   All calls on a device share the buffer: nothing needs clearing between calls, but calls
  *   that may overlap on the GPU (other streams, other host threads) race and must be
  *   serialised by the caller. */

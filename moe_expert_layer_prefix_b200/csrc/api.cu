@@ -17,7 +17,6 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<int> g_tile_mode{0};
 
 constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices] = {};
 int g_sms[kMaxDevices] = {};
 std::mutex g_mu;
 
@@ -33,15 +32,19 @@ void count_launch(int n) { g_launches.fetch_add(static_cast<uint64_t>(n)); }
 int gemm_tile_mode() { return g_tile_mode.load(); }
 
 int* device_error_word() {
-  const int d = current_device();
-  if (d < 0 || d >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (g_err_ptr[d] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
-    g_err_ptr[d] = static_cast<int*>(p);
-  }
-  return g_err_ptr[d];
+  // looked up on every call (cheap): a cached address would go stale after a device reset
+  // or in another context on the same device
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+moe_status check_dispatch_shapes(int T, int H, int E, int k) {
+  if (T < 1 || H < 128 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
+  if (H % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (E > 1024 || k > 32 || k > E || static_cast<long long>(T) * k > INT32_MAX)
+    return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
 }
 
 int num_sms() {
@@ -81,12 +84,7 @@ inline moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK 
 // Slot indices t*k + j are 32-bit on the device.
 inline bool slots_fit(int T, int k) { return static_cast<long long>(T) * k <= INT32_MAX; }
 
-moe_status check_shapes(int T, int H, int E, int k) {
-  if (T < 1 || H < 128 || E < 1 || k < 1) return MOE_ERR_INVALID_ARG;
-  if (H % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  if (E > 1024 || k > 32 || k > E || !slots_fit(T, k)) return MOE_ERR_UNSUPPORTED;
-  return MOE_OK;
-}
+moe_status check_shapes(int T, int H, int E, int k) { return check_dispatch_shapes(T, H, E, k); }
 
 moe_status check_weights(const moe_weights* W, int need_act) {
   if (W == nullptr || W->w1 == nullptr || W->w2 == nullptr) return MOE_ERR_INVALID_ARG;

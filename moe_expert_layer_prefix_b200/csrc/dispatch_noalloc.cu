@@ -10,15 +10,15 @@
 //
 // The buffer is a file-scope __device__ array, so every GPU that loads the library holds
 // it (kNoAllocScratchBytes) until the process exits.  Host code cannot use the array's name
-// as a device address; the first call on each device looks the address up with
-// cudaGetSymbolAddress while that device is current and caches it.
+// as a device address: every call looks the address up with cudaGetSymbolAddress while
+// the caller's device is current (the lookup is cheap, and nothing is cached, so a reset
+// device or a new context never sees a stale address).  The first call on a device also
+// loads the library's module there; make it before any stream capture.
 //
 // All calls on a device share the one buffer.  Dispatch overwrites every scratch word it
 // later reads, so nothing needs clearing between calls, but calls whose executions overlap
 // on the GPU (different streams, or different host threads) race on the buffer and must
 // be serialised by the caller.
-#include <mutex>
-
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,26 +28,6 @@ constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB per device
 
 static __device__ __align__(256) unsigned char g_dispatch_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
-void* g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Device address of g_dispatch_scratch on the current device (looked up once per device).
-moe_status scratch_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_dispatch_scratch) != cudaSuccess || p == nullptr)
-      return MOE_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
-  return MOE_OK;
-}
-
 }  // namespace
 
 extern "C" moe_status moe_dispatch_noalloc(const void* x, const float* x_scales, int act, int T,
@@ -55,11 +35,14 @@ extern "C" moe_status moe_dispatch_noalloc(const void* x, const float* x_scales,
                                            void* x_perm, float* x_perm_scales,
                                            int32_t* expert_offsets, int32_t* perm_src,
                                            int32_t* slot_of, cudaStream_t stream) {
-  if (T < 1 || E < 1 || E > 1024) return MOE_ERR_INVALID_ARG;
+  // the shape checks of moe_dispatch come first, so both entry points give the same status
+  // for a shape neither supports; only then is the buffer's size the deciding limit
+  const moe_status shapes = moe::check_dispatch_shapes(T, H, E, k);
+  if (shapes != MOE_OK) return shapes;
   if (moe::dispatch_ws_bytes(T, E) > kNoAllocScratchBytes) return MOE_ERR_WORKSPACE;
   void* scratch = nullptr;
-  const moe_status st = scratch_address(&scratch);
-  if (st != MOE_OK) return st;
+  if (cudaGetSymbolAddress(&scratch, g_dispatch_scratch) != cudaSuccess || scratch == nullptr)
+    return MOE_ERR_CUDA;
   return moe_dispatch(x, x_scales, act, T, H, E, k, topk_idx, x_perm, x_perm_scales,
                       expert_offsets, perm_src, slot_of, scratch, kNoAllocScratchBytes, stream);
 }

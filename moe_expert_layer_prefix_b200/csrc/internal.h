@@ -8,6 +8,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
 void count_launch(int n = 1);
@@ -111,5 +113,9 @@ int gemm_tile_mode();
 // m-blocks).  allow_pair = false where only single-CTA shapes exist (the persistent kernel).
 int gemm_tile_shape(int act, int S, int E, bool allow_pair);       // 0 automatic, 1 single-CTA tiles, 2 CTA-pair tiles
 int num_sms();
+
+// Shape checks shared by the dispatch entry points (and the layer-level calls): T, H, E, k
+// within the supported ranges.  Returns MOE_OK, MOE_ERR_INVALID_ARG or MOE_ERR_UNSUPPORTED.
+moe_status check_dispatch_shapes(int T, int H, int E, int k);
 
 }  // namespace moe
