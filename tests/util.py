@@ -83,9 +83,46 @@ def parity_err(got: np.ndarray, ref: np.ndarray, fmt: str, rms: float | None = N
     return float(np.max(excess)) / max(rms, 1e-30), rel_l2
 
 
+def raw_err(got: np.ndarray, ref: np.ndarray, rms: float | None = None) -> float:
+    """The tolerance figure as stated for the layer, with no allowance of any kind:
+    max |got - ref| / rms(ref)."""
+    ref = np.asarray(ref, np.float64)
+    if rms is None:
+        rms = float(np.sqrt(np.mean(ref ** 2)))
+    return float(np.max(np.abs(np.asarray(got, np.float64) - ref))) / max(rms, 1e-30)
+
+
 def assert_parity(got, ref, fmt, tol, rms=None):
     mx, l2 = parity_err(got, ref, fmt, rms)
-    assert mx <= tol and l2 <= tol, f"max-excess/rms={mx:.3e} rel-L2={l2:.3e} tol={tol}"
+    raw = raw_err(got, ref, rms)
+    assert mx <= tol and l2 <= tol, (f"max-excess/rms={mx:.3e} rel-L2={l2:.3e} tol={tol} "
+                                     f"(raw max|gpu-oracle|/rms(oracle)={raw:.3e})")
+    return mx, l2, raw
+
+
+# Per-operation relative error of an fp32 accumulation: 2^-23 covers round-to-nearest and
+# truncation alike, whatever order the tensor cores or the CUDA cores add in.
+FP32_ACC_EPS = 2.0 ** -23
+
+
+def fp32_sum_bound(abs_terms_sum: np.ndarray, K: int) -> np.ndarray:
+    """Bound on |fp32 sum - exact sum| of K exactly representable products whose absolute
+    values sum to abs_terms_sum (the classic (K - 1) * eps * sum|a_i b_i| bound of recursive
+    summation, valid for any association order)."""
+    return (K - 1) * FP32_ACC_EPS * abs_terms_sum
+
+
+def assert_within_bound(got, ref, bound, fmt, what):
+    """|got - ref| <= one storage ulp at |ref| + bound, plus the bound itself, element by
+    element: got is ref computed in fp32 (error <= bound) and then rounded to `fmt`, while
+    ref is rounded from fp64, so the two roundings can fall one ulp apart on top of the
+    fp32 error."""
+    ref = np.asarray(ref, np.float64)
+    lim = store_ulp(np.abs(ref) + bound, fmt) + bound
+    d = np.abs(np.asarray(got, np.float64) - ref)
+    bad = d > lim
+    assert not bad.any(), (f"{what}: {int(bad.sum())} of {d.size} elements beyond the fp32 "
+                           f"accumulation bound; worst |d|/lim = {float(np.max(d / np.maximum(lim, 1e-300))):.3f}")
 
 
 TOL = {"f32": 1e-4, "bf16": 1e-2, "e4m3": 3e-2}
