@@ -312,9 +312,34 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
  * Returns MOE_OK, or the first recorded failure with *site (may be NULL) set to the code
  * location that recorded it, or MOE_ERR_CUDA if the synchronisation itself failed.
  * Recorded failures: MOE_ERR_TIMEOUT at a bounded wait (sites 101-106: GEMM pipeline
- * barriers; 201: the persistent kernel's grid barrier), MOE_ERR_UNSUPPORTED at site 301
- * (an fp32 block scale that is not a positive normal power of two). */
+ * barriers; 201: the persistent kernel's grid barrier; 901: the self-test's mbarrier),
+ * MOE_ERR_UNSUPPORTED at site 301 (an fp32 block scale that is not a positive normal power
+ * of two).  The wait limit (moe_set_wait_limit) is kept. */
 moe_status moe_get_device_error(cudaStream_t stream, int* site);
+
+/* Limit of every bounded wait in the library's kernels (mbarrier waits of the GEMM
+ * pipeline and its drains, the persistent kernel's grid barriers), in SM clock cycles, for
+ * the calling thread's current device (call once per device; it holds for every later
+ * launch on that device, from any host thread).  0 restores the default of 2e9 cycles
+ * (about one second at the B200's boost clock; legitimate waits take microseconds).  A wait
+ * that runs past the limit records MOE_ERR_TIMEOUT and its site in the device error word
+ * and its kernel returns without finishing the work, leaving the context usable.
+ * Synchronous (a 8-byte copy to the device).  Returns MOE_ERR_INVALID_ARG for cycles < 0,
+ * MOE_ERR_CUDA if the copy fails. */
+moe_status moe_set_wait_limit(long long cycles);
+
+/* Self-test of the bounded waits (failure detection; the source pages have no counterpart).
+ * Launches a kernel whose wait can never be satisfied, by construction:
+ *   MOE_SELFTEST_MBARRIER      one CTA waits on an mbarrier that nothing arrives on;
+ *                              records MOE_ERR_TIMEOUT at site 901
+ *   MOE_SELFTEST_GRID_BARRIER  every CTA of a cooperative grid (one per SM) arrives at a
+ *                              grid barrier expecting one arrival more than the grid has;
+ *                              records MOE_ERR_TIMEOUT at site 201
+ * The kernel returns once the wait limit has passed; read the result with
+ * moe_get_device_error.  Nothing traps, faults or waits without a limit.  Returns
+ * MOE_ERR_INVALID_ARG for another kind, MOE_ERR_CUDA if the launch fails. */
+enum { MOE_SELFTEST_MBARRIER = 0, MOE_SELFTEST_GRID_BARRIER = 1 };
+moe_status moe_selftest_wait(int kind, cudaStream_t stream);
 
 /* Static string naming a status code. */
 const char* moe_status_string(int status);

@@ -35,7 +35,8 @@ EXPORTS = ("moe_route", "moe_dispatch", "moe_expert_linear1", "moe_expert_linear
            "moe_fused_ffn", "moe_combine", "moe_forward", "moe_workspace_size",
            "moe_get_device_error", "moe_status_string", "moe_launch_count",
            "moe_dispatch_noalloc", "moe_set_gemm_tiles", "moe_dispatch_quant", "moe_route_ex",
-           "moe_forward_ex", "moe_transpose_experts", "moe_expert_backward")
+           "moe_forward_ex", "moe_transpose_experts", "moe_expert_backward",
+           "moe_set_wait_limit", "moe_selftest_wait")
 
 _P, _I, _Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 
@@ -91,6 +92,8 @@ _get_err = _sig("moe_get_device_error", _I, [_P, ctypes.POINTER(ctypes.c_int)])
 _status_string = _sig("moe_status_string", ctypes.c_char_p, [_I])
 _launch_count = _sig("moe_launch_count", ctypes.c_uint64, [])
 _set_tiles = _sig("moe_set_gemm_tiles", _I, [_I])
+_set_wait_limit = _sig("moe_set_wait_limit", _I, [ctypes.c_longlong])
+_selftest_wait = _sig("moe_selftest_wait", _I, [_I, _P])
 
 
 class MoeError(RuntimeError):
@@ -114,6 +117,21 @@ def moe_set_gemm_tiles(mode="auto"):
     """Process-wide tile shape of the expert GEMMs: 'auto', 'single' (128-row tiles, one
     CTA), 'pair' (256-row tiles, 2-CTA cluster) or 'small' (32-row tiles, one CTA)."""
     _check(_set_tiles(TILES[mode] if isinstance(mode, str) else mode), "moe_set_gemm_tiles")
+
+
+def moe_set_wait_limit(cycles=0):
+    """Limit of every bounded wait in the library's kernels on the current device, in SM
+    clock cycles (0: the default, about one second)."""
+    _check(_set_wait_limit(int(cycles)), "moe_set_wait_limit")
+
+
+SELFTEST = {"mbarrier": 0, "grid_barrier": 1}
+
+
+def moe_selftest_wait(kind, stream=None):
+    """Launch a kernel whose bounded wait runs out by construction ('mbarrier' or
+    'grid_barrier'); read the recorded timeout with moe_get_device_error()."""
+    _check(_selftest_wait(SELFTEST[kind], _stream(stream)), "moe_selftest_wait")
 
 
 def _ptr(t):

@@ -1,6 +1,7 @@
 // C ABI of libmoe.so: argument checking, workspace carving and launch sequencing.
 // Every computation happens in the kernels of the other translation units.
 #include <atomic>
+#include <cstddef>
 #include <climits>
 #include <mutex>
 
@@ -9,8 +10,15 @@
 
 namespace moe {
 
-// Per-device error word {status, site}, written by kernels whose waits are bounded.
-__device__ int g_error_word[2];
+// Per-device control block: the error word {status, site} that kernels whose waits are
+// bounded write, followed by the wait limit they read (SM clock cycles).
+struct DevCtl {
+  int status;
+  int site;
+  long long wait_limit;
+};
+static_assert(offsetof(DevCtl, wait_limit) == 8, "kernels read the limit at err + 2");
+__device__ DevCtl g_error_word = {0, 0, kWaitLimitCycles};
 
 namespace {
 std::atomic<uint64_t> g_launches{0};
@@ -135,6 +143,15 @@ const char* moe_status_string(int status) {
 
 uint64_t moe_launch_count(void) { return g_launches.load(); }
 
+moe_status moe_set_wait_limit(long long cycles) {
+  if (cycles < 0) return MOE_ERR_INVALID_ARG;
+  const long long v = cycles == 0 ? kWaitLimitCycles : cycles;
+  if (cudaMemcpyToSymbol(g_error_word, &v, sizeof(v), offsetof(DevCtl, wait_limit)) !=
+      cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 moe_status moe_set_gemm_tiles(int mode) {
   if (mode < 0 || mode > 3) return MOE_ERR_INVALID_ARG;
   g_tile_mode.store(mode);
@@ -186,7 +203,7 @@ moe_status moe_get_device_error(cudaStream_t stream, int* site) {
   int host[2] = {0, 0};
   if (cudaMemcpyFromSymbol(host, g_error_word, sizeof(host)) != cudaSuccess) return MOE_ERR_CUDA;
   if (host[0] != 0) {
-    const int zero[2] = {0, 0};
+    const int zero[2] = {0, 0};  // status and site only; the wait limit stays
     if (cudaMemcpyToSymbol(g_error_word, zero, sizeof(zero)) != cudaSuccess) return MOE_ERR_CUDA;
   }
   if (site) *site = host[1];

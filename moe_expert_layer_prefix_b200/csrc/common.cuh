@@ -25,14 +25,24 @@ enum Site : int {
   SITE_GEMM_DRAIN = 106,     // loader draining its in-flight copies after an abort
   SITE_GRID_BARRIER = 201,   // persistent kernel waiting at a grid-wide barrier
   SITE_SCALE_FORMAT = 301,   // an fp32 block scale that is not a positive normal power of two
+  SITE_SELFTEST_MBAR = 901,  // self-test: a wait on an mbarrier nothing ever arrives on
 };
 
 __device__ __forceinline__ void report_error(int* err, int code, int site) {
   if (err != nullptr && atomicCAS(err, 0, code) == 0) atomicExch(err + 1, site);
 }
 
-// About one second at the B200's boost clock; legitimate waits are microseconds.
+// The device control block the error pointer of every waiting kernel points at:
+// {status, site, wait limit in SM clock cycles (64-bit, 8-byte aligned)}.  The limit is
+// process-wide per device (moe_set_wait_limit); about one second at the B200's boost clock
+// by default, while legitimate waits are microseconds.
 constexpr long long kWaitLimitCycles = 2000000000LL;
+
+__device__ __forceinline__ long long wait_limit(const int* err) {
+  if (err == nullptr) return kWaitLimitCycles;
+  const long long v = *reinterpret_cast<const volatile long long*>(err + 2);
+  return v > 0 ? v : kWaitLimitCycles;
+}
 
 // ---------------------------------------------------------------------------------------
 // small utilities
@@ -110,11 +120,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
                                           volatile int* abort) {
   if (mbar_try_wait_scoped<kCluster>(bar, parity)) return true;
   const long long t0 = clock64();
+  const long long limit = wait_limit(err);
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_scoped<kCluster>(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > limit) {
         report_error(err, MOE_ERR_TIMEOUT, site);
         *abort = 1;
         return false;
@@ -421,8 +432,9 @@ __device__ __forceinline__ float exp2i(int n) {  // 2^n for -126 <= n <= 127
 
 // ---------------------------------------------------------------------------------------
 // grid-wide barrier for co-resident (cooperative) grids: bar[0] arrivals, bar[1] generation
-// (both zero before the launch).  Bounded: gives up after kWaitLimitCycles, records
-// MOE_ERR_TIMEOUT at SITE_GRID_BARRIER and returns false.
+// (both zero before the launch).  `expected` arrivals complete it (the grid's CTA count).
+// Bounded: gives up after the wait limit, records MOE_ERR_TIMEOUT at SITE_GRID_BARRIER and
+// returns false (in every thread of the CTA).
 // ---------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
@@ -430,7 +442,7 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   return v;
 }
 
-__device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {
+__device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expected) {
   __syncthreads();
   __shared__ int ok_s;
   if (threadIdx.x == 0) {
@@ -438,14 +450,15 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {
     const uint32_t gen = ld_acquire_gpu(bar + 1);
     __threadfence();
     const uint32_t arrived = atomicAdd(bar, 1u);
-    if (arrived == gridDim.x - 1) {
+    if (arrived == expected - 1) {
       atomicExch(bar, 0u);
       __threadfence();
       atomicAdd(bar + 1, 1u);
     } else {
       const long long t0 = clock64();
+      const long long limit = wait_limit(err);
       while (ld_acquire_gpu(bar + 1) == gen) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
           report_error(err, MOE_ERR_TIMEOUT, SITE_GRID_BARRIER);
           ok = 0;
           break;
@@ -457,6 +470,10 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {
   }
   __syncthreads();
   return ok_s != 0;
+}
+
+__device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {
+  return grid_sync(bar, err, gridDim.x);
 }
 
 }  // namespace moe

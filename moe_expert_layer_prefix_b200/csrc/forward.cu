@@ -83,86 +83,90 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   int32_t* soffs = reinterpret_cast<int32_t*>(scratch + nwarps * kMaxE * 4 + 32 * 33 * 4);
   int32_t* wsum = soffs + 1028;
 
-  // 1. route: one warp per token
-  if (p.E <= 256) {
-    for (int t = gw; t < p.T; t += GW)
-      route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
-                     p.n_group, p.topk_group, p.scale);
-  } else {
-    for (int t = gw; t < p.T; t += GW)
-      route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
-                      p.n_group, p.topk_group, p.scale);
-  }
-  grid_sync(p.bar, p.err);
-
-  // 2. per-chunk expert counts
-  for (int c = gw; c < p.C; c += GW) hist_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, lane, p.cnt);
-  grid_sync(p.bar, p.err);
-
-  // 3. per-expert scans over the chunks (32 experts per CTA pass)
-  for (int g = blockIdx.x; g < (p.E + 31) / 32; g += gridDim.x)
-    scan_group(p.cnt, p.E, p.C, p.totals, g, nwarps, warp, lane, part);
-  grid_sync(p.bar, p.err);
-
-  // 4. expert offsets (every CTA keeps its own copy; CTA 0 publishes them)
-  offsets_from_totals(p.totals, p.E, soffs, wsum);
-  if (blockIdx.x == 0)
-    for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.offsets[e] = soffs[e];
-
-  // 5. slots and permutation (one warp per 32-token chunk)
-  for (int c = gw; c < p.C; c += GW)
-    assign_slots_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, p.cnt, soffs, p.perm_src, p.slot_of,
-                       lane);
-  grid_sync(p.bar, p.err);
-
-  // 6. row copies x -> x_perm (one warp per token), quantising BF16 rows when asked
-  if (p.quant_x) {
-    for (int t = gw; t < p.T; t += GW)
-      quant_copy_token_rows(static_cast<const __nv_bfloat16*>(p.x), p.H, p.slot_of, t, p.k,
-                            static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
-  } else {
-    for (int t = gw; t < p.T; t += GW)
-      copy_token_rows(static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes, p.H / 128,
-                      p.slot_of, t, p.k, static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
-  }
-  fence_proxy_async_global();  // x_perm is read by TMA next
-  grid_sync(p.bar, p.err);
-
-  // 7. linear-1 + SwiGLU + requantisation
-  Pipe pipe;
-  gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l1.n_tiles);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  gemm_phase<1, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
-  fence_proxy_async_global();  // h is read by TMA next
-  grid_sync(p.bar, p.err);
-
-  // 8. linear-2
-  gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l2.n_tiles);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
-  grid_sync(p.bar, p.err);
-
-  // 9. combine.  With only 8 warps per SM here, a warp keeps four 16-byte loads per lane and
-  //    source row in flight and takes a whole token when there are tokens enough for every
-  //    warp; fewer tokens are split into 512-column chunks with two loads in flight (the
-  //    faster of the shapes measured on the V3, skewed and decode layers).
-  if (p.T >= 2 * GW) {
-    for (int t = gw; t < p.T; t += GW)
-      combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
-  } else {
-    const int nc = combine_chunks<2>(p.H);
-    const int width = nc == 1 ? p.H / 8 : 64;
-    const long items = static_cast<long>(p.T) * nc;
-    for (long it = gw; it < items; it += GW) {
-      const int t = static_cast<int>(it / nc), c = static_cast<int>(it % nc);
-      combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
-                              (c + 1) * width);
+  // A grid barrier that timed out (recorded in the error word) ends the phases for this
+  // CTA: it releases TMEM and returns; the other CTAs give up at their next barrier.
+  do {
+    // 1. route: one warp per token
+    if (p.E <= 256) {
+      for (int t = gw; t < p.T; t += GW)
+        route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
+                       p.n_group, p.topk_group, p.scale);
+    } else {
+      for (int t = gw; t < p.T; t += GW)
+        route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
+                        p.n_group, p.topk_group, p.scale);
     }
-  }
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 2. per-chunk expert counts
+    for (int c = gw; c < p.C; c += GW) hist_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, lane, p.cnt);
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 3. per-expert scans over the chunks (32 experts per CTA pass)
+    for (int g = blockIdx.x; g < (p.E + 31) / 32; g += gridDim.x)
+      scan_group(p.cnt, p.E, p.C, p.totals, g, nwarps, warp, lane, part);
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 4. expert offsets (every CTA keeps its own copy; CTA 0 publishes them)
+    offsets_from_totals(p.totals, p.E, soffs, wsum);
+    if (blockIdx.x == 0)
+      for (int e = threadIdx.x; e <= p.E; e += blockDim.x) p.offsets[e] = soffs[e];
+
+    // 5. slots and permutation (one warp per 32-token chunk)
+    for (int c = gw; c < p.C; c += GW)
+      assign_slots_chunk(mask, p.topk_idx, p.T, p.E, p.k, c, p.cnt, soffs, p.perm_src, p.slot_of,
+                         lane);
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 6. row copies x -> x_perm (one warp per token), quantising BF16 rows when asked
+    if (p.quant_x) {
+      for (int t = gw; t < p.T; t += GW)
+        quant_copy_token_rows(static_cast<const __nv_bfloat16*>(p.x), p.H, p.slot_of, t, p.k,
+                              static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
+    } else {
+      for (int t = gw; t < p.T; t += GW)
+        copy_token_rows(static_cast<const uint8_t*>(p.x), p.x_scales, p.row_bytes, p.H / 128,
+                        p.slot_of, t, p.k, static_cast<uint8_t*>(p.x_perm), p.x_perm_scales, lane);
+    }
+    fence_proxy_async_global();  // x_perm is read by TMA next
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 7. linear-1 + SwiGLU + requantisation
+    Pipe pipe;
+    gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l1.n_tiles);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    gemm_phase<1, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
+    fence_proxy_async_global();  // h is read by TMA next
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 8. linear-2
+    gemm_prefix<1, kTm>(sm, p.offsets, p.E, p.l2.n_tiles);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 9. combine.  With only 8 warps per SM here, a warp keeps four 16-byte loads per lane and
+    //    source row in flight and takes a whole token when there are tokens enough for every
+    //    warp; fewer tokens are split into 512-column chunks with two loads in flight (the
+    //    faster of the shapes measured on the V3, skewed and decode layers).
+    if (p.T >= 2 * GW) {
+      for (int t = gw; t < p.T; t += GW)
+        combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
+    } else {
+      const int nc = combine_chunks<2>(p.H);
+      const int width = nc == 1 ? p.H / 8 : 64;
+      const long items = static_cast<long>(p.T) * nc;
+      for (long it = gw; it < items; it += GW) {
+        const int t = static_cast<int>(it / nc), c = static_cast<int>(it % nc);
+        combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
+                                (c + 1) * width);
+      }
+    }
+  } while (0);
 
   tc_fence_before();
   __syncthreads();

@@ -385,8 +385,9 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           const int stage = static_cast<int>((it - i) % kStages);
           const uint32_t phase = ((it - i) / kStages) & 1u;
           const long long t0 = clock64();
+          const long long limit = wait_limit(p.err);
           while (!mbar_try_wait_scoped<kPair>(&ss.full[stage], phase)) {
-            if (clock64() - t0 > kWaitLimitCycles) {
+            if (clock64() - t0 > limit) {
               report_error(p.err, MOE_ERR_TIMEOUT, SITE_GEMM_DRAIN);
               break;
             }
@@ -496,8 +497,9 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
         if constexpr (kPair) tc_commit_pair(&ss.drain, 0x1);
         else tc_commit(&ss.drain);
         const long long t0 = clock64();
+        const long long limit = wait_limit(p.err);
         while (!mbar_try_wait_scoped<kPair>(&ss.drain, 0)) {
-          if (clock64() - t0 > kWaitLimitCycles) break;
+          if (clock64() - t0 > limit) break;
         }
       }
     }

@@ -107,6 +107,9 @@ struct ForwardArgs {
 };
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s);
 
+// Self-test kernels whose bounded waits run out by construction (selftest.cu).
+cudaError_t launch_wait_selftest(int kind, int* err, cudaStream_t s);
+
 int* device_error_word();   // device address of the calling device's error word
 int gemm_tile_mode();
 // Tile shape for a grouped GEMM over S rows and E experts: 1 single, 2 pair, 3 small (32-row

@@ -81,6 +81,11 @@ def test_argument_errors_need_no_gpu():
     assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
 
 
+def test_wait_limit_and_selftest_arguments_checked_before_any_device_call():
+    assert M.moe_status_string(M._set_wait_limit(-1)) == "MOE_ERR_INVALID_ARG"
+    assert M.moe_status_string(M._selftest_wait(7, None)) == "MOE_ERR_INVALID_ARG"
+
+
 def test_slot_count_beyond_32_bits_is_refused_before_launch():
     # slot indices t*k + j are 32-bit on the device: T*k > 2^31 - 1 is refused, and sizes
     # to zero, on the host (the dummy addresses are never dereferenced)
