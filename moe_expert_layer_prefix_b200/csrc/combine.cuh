@@ -69,6 +69,9 @@ __device__ __forceinline__ void combine_token(const void* __restrict__ y,
       }
 #pragma unroll
       for (int jj = 0; jj < kJ; ++jj) {
+        // rows past the token's k are not loaded at all (k = 2 would otherwise re-read a
+        // row six times per pass)
+        if (j0 + jj >= k) break;  // warp-uniform
         const uint4* row = y4 + static_cast<size_t>(slot[jj]) * row_words;
 #pragma unroll
         for (int p = 0; p < kV; ++p)

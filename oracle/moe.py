@@ -311,9 +311,11 @@ def forward(L: Layer, return_all: bool = False):
                 perm_src=perm_src, slot_of=slot_of, y=y, h=h_all)
 
 
-def forward_tokens(L: Layer, tokens) -> np.ndarray:
+def forward_tokens(L: Layer, tokens, return_y: bool = False):
     """out rows for the listed tokens only (routing is per token, so no other token is
-    needed).  Work is grouped by expert so each expert's weights are dequantised once."""
+    needed).  Work is grouped by expert so each expert's weights are dequantised once.
+    With return_y, also the stored y rows the combine sums, [n, k, H] in rank order, and
+    the gates as stored (fp32), [n, k]."""
     tokens = np.asarray(tokens, dtype=np.int64)
     idx, w = route(L.logits[tokens], L.bias, L.k, L.score, L.renorm)
     w32 = w.astype(np.float32).astype(np.float64)
@@ -329,7 +331,10 @@ def forward_tokens(L: Layer, tokens) -> np.ndarray:
     for r in range(tokens.size):
         for j in range(L.k):
             out[r] = out[r] + w32[r, j] * acc[r][j]
-    return _store_y(out, L.act)
+    out = _store_y(out, L.act)
+    if return_y:
+        return out, np.array([[acc[r][j] for j in range(L.k)] for r in range(tokens.size)]), w32
+    return out
 
 
 def ffn_slots(L: Layer, slots, perm_src, offsets) -> np.ndarray:
