@@ -23,6 +23,7 @@ enum Site : int {
   SITE_GEMM_ACC_EMPTY = 104, // MMA issuer waiting for the epilogue to drain TMEM
   SITE_GEMM_SF_EMPTY = 105,  // scale-factor loader waiting for a free smem stage
   SITE_GEMM_DRAIN = 106,     // loader draining its in-flight copies after an abort
+  SITE_GEMM_AMAX = 107,      // linear-1 epilogue waiting for the other half's row amax
   SITE_GRID_BARRIER = 201,   // persistent kernel waiting at a grid-wide barrier
   SITE_SCALE_FORMAT = 301,   // an fp32 block scale that is not a positive normal power of two
   SITE_SELFTEST_MBAR = 901,  // self-test: a wait on an mbarrier nothing ever arrives on
@@ -444,9 +445,8 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
 
 __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expected) {
   __syncthreads();
-  __shared__ int ok_s;
+  int ok = 1;  // thread 0's verdict, shared through the closing barrier (no shared memory)
   if (threadIdx.x == 0) {
-    int ok = 1;
     const uint32_t gen = ld_acquire_gpu(bar + 1);
     __threadfence();
     const uint32_t arrived = atomicAdd(bar, 1u);
@@ -466,10 +466,8 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expe
       }
     }
     __threadfence();
-    ok_s = ok;
   }
-  __syncthreads();
-  return ok_s != 0;
+  return __syncthreads_and(ok) != 0;
 }
 
 __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {

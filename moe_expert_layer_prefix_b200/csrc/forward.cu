@@ -149,13 +149,12 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
     if (!grid_sync(p.bar, p.err)) break;
 
-    // 9. combine.  With only 8 warps per SM here, a warp keeps four 16-byte loads per lane and
-    //    source row in flight and takes a whole token when there are tokens enough for every
-    //    warp; fewer tokens are split into 512-column chunks with two loads in flight (the
-    //    faster of the shapes measured on the V3, skewed and decode layers).
+    // 9. combine.  A warp keeps two 16-byte loads per lane and source row in flight and
+    //    takes a whole token when there are tokens enough for every warp; fewer tokens are
+    //    split into 512-column chunks.
     if (p.T >= 2 * GW) {
       for (int t = gw; t < p.T; t += GW)
-        combine_token<false, 4>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
+        combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
     } else {
       const int nc = combine_chunks<2>(p.H);
       const int width = nc == 1 ? p.H / 8 : 64;

@@ -27,10 +27,14 @@
 //               into a 16-slot shared-memory ring with asynchronous 4-byte copies (cp.async)
 //   warp 3      scale converter: UE8M0 bytes in the layout tcgen05.cp reads, then signals the
 //               (leader's) slot barriers; before each GEMM phase it also builds the tile list
-//   warps 4..7  epilogue: tcgen05.ld of the accumulator (warp i reads TMEM lanes 32i..32i+31,
-//               one output row per thread), SwiGLU + BF16 / E4M3 requantisation (linear-1)
-//               or BF16 conversion (linear-2); 16-byte global stores, for linear-2 after
-//               lane pairs swap chunks so that every store writes whole 32-byte sectors
+//   warps 4..11 epilogue: two warps per TMEM lane quadrant (warp w reads lanes
+//               32(w%4)..+31, one output row per thread), each taking half of the tile's
+//               columns, so that the accumulator is read out in a quarter of the time and
+//               handed back to the MMA issuer before any arithmetic: SwiGLU + BF16 / E4M3
+//               requantisation (linear-1; the two halves of a row exchange their partial
+//               amax through shared memory) or BF16 conversion (linear-2); 16-byte global
+//               stores, for linear-2 after lane pairs swap chunks so that every store writes
+//               whole 32-byte sectors
 //
 // linear-1 tiles take B rows [n*128, n*128+128) (gate) and [I + n*128, ...) (up), so the
 // accumulator holds gate in columns 0..127 and up in 128..255 and each tile yields 128 h
@@ -65,7 +69,8 @@ constexpr int kSfbCol = 260;       // ... SFA (4 columns) then SFB (8 columns)
 constexpr int kSfSetCols = 12;
 constexpr int kSfSets = 4;         // rotated (per copy) so that a copy never overwrites the
                                    // scales an earlier k-step's MMAs may still be reading
-constexpr int kThreads = 256;
+constexpr int kEpiWarps = 8;       // two warps per TMEM lane quadrant, one per column half
+constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
 constexpr int kSfSlots = 16;       // scale-factor ring, decoupled from (and deeper than) the A/B ring
@@ -94,6 +99,10 @@ struct SharedState {
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
+  uint64_t amax_bar[4];         // linear-1 E4M3 epilogue: both column halves of a quadrant
+                                // have published their row's scale exponent
+  int8_t ecode[2][2][kBM];      // [tile parity][column half][row of the tile]: the scale
+                                // exponent of the half's amax (kNoExp for an all-zero half)
   uint32_t tmem_base;
   int abort;
   int total_tiles;
@@ -218,6 +227,7 @@ struct Pipe {
   uint32_t tiles = 0;    // MMA issuer / epilogue: accumulator uses
   uint32_t sf_it = 0;    // scale loader / converter: k-steps staged
   uint32_t sf_grp = 0;   // MMA issuer: groups of 4 k-steps whose scales were copied to TMEM
+  uint32_t hq = 0;       // epilogue: linear-1 tiles requantised to E4M3 (amax exchanges)
 };
 
 // Shared-memory carve-up (1024-byte aligned; identical offsets in both CTAs of a pair).
@@ -257,8 +267,9 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
       mbar_init(&ss.sf_empty[s], 1);
     }
     mbar_init(&ss.acc_full, 1);
-    mbar_init(&ss.acc_empty, 4 * kCta);
+    mbar_init(&ss.acc_empty, kEpiWarps * kCta);
     mbar_init(&ss.drain, 1);
+    for (int q = 0; q < 4; ++q) mbar_init(&ss.amax_bar[q], 64);  // every lane of both halves
     ss.abort = 0;
     fence_barrier_init();
     for (int i = 0; i < ntmaps; ++i) tma_prefetch_desc(tmaps + i);
@@ -659,9 +670,10 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
-    const int q = warp - 4;  // TMEM lane quadrant
+    const int q = warp & 3;             // TMEM lane quadrant (the warp's 32 rows)
+    const int half = (warp - 4) >> 2;   // column half of the accumulator this warp reads
     const uint32_t trow = tmem + (static_cast<uint32_t>(q * 32) << 16);
-    uint32_t tiles = pipe.tiles;
+    uint32_t tiles = pipe.tiles, hq = pipe.hq;
     const uint32_t acc_empty_lead = mapa_shared(smem_u32(&ss.acc_empty), 0);
     for (int t = cid; t < total && !*abort; t += ncl) {
       const uint32_t acc_phase = tiles & 1u;
@@ -677,113 +689,109 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       const bool valid = q * 32 + lane < kTm && row < tile.m_end;
       // rows of this warp that exist (the tile's rows of this CTA, up to the expert's end)
       const int rows_ok = min(kTm - q * 32, tile.m_end - row0);
+      // the warp's 128 accumulator columns: linear-1 gate [64h, 64h+64) and up
+      // [128 + 64h, +64); linear-2 [128h, 128h + 128)
+      uint32_t d[128];
       if constexpr (kSwiGLU) {
+        tmem_ld32(trow + kAccCol + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(d));
+        tmem_ld32(trow + kAccCol + 64 * half + 32, *reinterpret_cast<uint32_t(*)[32]>(d + 32));
+        tmem_ld32(trow + kAccCol + 128 + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(d + 64));
+        tmem_ld32(trow + kAccCol + 160 + 64 * half, *reinterpret_cast<uint32_t(*)[32]>(d + 96));
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(trow + kAccCol + 128 * half + 32 * c,
+                    *reinterpret_cast<uint32_t(*)[32]>(d + 32 * c));
+      }
+      tmem_ld_wait();
+      // the accumulator is in registers: hand TMEM back before any arithmetic
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
+        else mbar_arrive(&ss.acc_empty);
+      }
+      if constexpr (kSwiGLU) {
+        float h[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          h[i] = silu_mul(__uint_as_float(d[i]), __uint_as_float(d[64 + i]));
         if constexpr (kOutE4M3) {
-          float h[128];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t g[32], u[32];
-            tmem_ld32(trow + kAccCol + 32 * c, g);
-            tmem_ld32(trow + kAccCol + 128 + 32 * c, u);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              h[32 * c + i] = silu_mul(__uint_as_float(g[i]), __uint_as_float(u[i]));
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
-          else mbar_arrive(&ss.acc_empty);
-        }
+          // one power-of-two scale per 128 h columns = the whole tile row: the two halves
+          // of the row exchange their partial amax
+          // of the row exchange the scale exponent of their partial amax: the exponent rule
+          // is monotonic in amax, so the row's exponent is the larger of the two (an
+          // all-zero half contributes nothing; an all-zero row takes scale 1)
           float amax = 0.0f;
 #pragma unroll
-          for (int i = 0; i < 128; ++i) amax = fmaxf(amax, fabsf(h[i]));
-          const int e = max(e4m3_scale_exponent(amax), -126);
+          for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(h[i]));
+          constexpr int kNoExp = -128;
+          const int own = amax > 0.0f ? max(e4m3_scale_exponent(amax), -126) : kNoExp;
+          const int slot = static_cast<int>(hq & 1u);
+          ss.ecode[slot][half][q * 32 + lane] = static_cast<int8_t>(own);
+          mbar_arrive(&ss.amax_bar[q]);
+          const bool got = mbar_wait(&ss.amax_bar[q], hq & 1u, p.err, SITE_GEMM_AMAX, abort);
+          ++hq;
+          if (!__all_sync(0xffffffffu, got)) break;
+          const int both = max(own, static_cast<int>(ss.ecode[slot][half ^ 1][q * 32 + lane]));
+          const int e = both == kNoExp ? 0 : both;
           const float inv = exp2i(-e);
           if (valid) {
             uint8_t* dst = static_cast<uint8_t*>(p.out) + static_cast<size_t>(row) * p.n_out +
-                           tile.nb * 128;
+                           tile.nb * 128 + 64 * half;
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int b = 16 * v + 4 * i;
+                const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+                    make_float2(h[b] * inv, h[b + 1] * inv), __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+                    make_float2(h[b + 2] * inv, h[b + 3] * inv), __NV_SATFINITE, __NV_E4M3);
+                w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+              }
+              reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            if (half == 0) p.out_scales[static_cast<size_t>(row) * (p.n_out / 128) + tile.nb] = exp2i(e);
+          }
+        } else {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
+                                                  static_cast<size_t>(row) * p.n_out +
+                                                  tile.nb * 128 + 64 * half);
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
               uint32_t w[4];
 #pragma unroll
               for (int i = 0; i < 4; ++i) {
-                const int b = 16 * v + 4 * i;
-                const __nv_fp8x2_storage_t lo =
-                    __nv_cvt_float2_to_fp8x2(make_float2(h[b] * inv, h[b + 1] * inv), __NV_SATFINITE, __NV_E4M3);
-                const __nv_fp8x2_storage_t hi =
-                    __nv_cvt_float2_to_fp8x2(make_float2(h[b + 2] * inv, h[b + 3] * inv), __NV_SATFINITE, __NV_E4M3);
-                w[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+                const __nv_bfloat162 b2 = __floats2bfloat162_rn(h[8 * v + 2 * i], h[8 * v + 2 * i + 1]);
+                w[i] = *reinterpret_cast<const uint32_t*>(&b2);
               }
-              reinterpret_cast<uint4*>(dst)[v] = make_uint4(w[0], w[1], w[2], w[3]);
+              dst[v] = make_uint4(w[0], w[1], w[2], w[3]);
             }
-            p.out_scales[static_cast<size_t>(row) * (p.n_out / 128) + tile.nb] = exp2i(e);
-          }
-        } else {
-          uint32_t w[64];  // 128 h values as BF16 pairs
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t g[32], u[32];
-            tmem_ld32(trow + kAccCol + 32 * c, g);
-            tmem_ld32(trow + kAccCol + 128 + 32 * c, u);
-            tmem_ld_wait();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                  silu_mul(__uint_as_float(g[2 * i]), __uint_as_float(u[2 * i])),
-                  silu_mul(__uint_as_float(g[2 * i + 1]), __uint_as_float(u[2 * i + 1])));
-              w[16 * c + i] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
-          else mbar_arrive(&ss.acc_empty);
-        }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) +
-                                                  static_cast<size_t>(row) * p.n_out + tile.nb * 128);
-#pragma unroll
-            for (int v = 0; v < 16; ++v)
-              dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
           }
         }
       } else {
-        // pack the whole row to BF16 in registers, hand TMEM back, then store
-        uint32_t w[kBN / 2];
+        // pack the warp's 128 columns of the row to BF16: chunk k = words 4k..4k+3 =
+        // columns nb*256 + 128*half + 8k .. + 8
+        uint32_t w[64];
 #pragma unroll
-        for (int c = 0; c < kBN / 32; c += 2) {  // two 32-column loads per wait
-          uint32_t d0[32], d1[32];
-          tmem_ld32(trow + kAccCol + 32 * c, d0);
-          tmem_ld32(trow + kAccCol + 32 * (c + 1), d1);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const __nv_bfloat162 b0 =
-                __floats2bfloat162_rn(__uint_as_float(d0[2 * i]), __uint_as_float(d0[2 * i + 1]));
-            const __nv_bfloat162 b1 =
-                __floats2bfloat162_rn(__uint_as_float(d1[2 * i]), __uint_as_float(d1[2 * i + 1]));
-            w[16 * c + i] = *reinterpret_cast<const uint32_t*>(&b0);
-            w[16 * (c + 1) + i] = *reinterpret_cast<const uint32_t*>(&b1);
-          }
+        for (int i = 0; i < 64; ++i) {
+          const __nv_bfloat162 b2 =
+              __floats2bfloat162_rn(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]));
+          w[i] = *reinterpret_cast<const uint32_t*>(&b2);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
-          else mbar_arrive(&ss.acc_empty);
-        }
-        // chunk k of the row = words 4k..4k+3 = columns nb*256 + 8k .. + 8
-        const int chunks_ok = min(kBN / 8, (p.n_out - tile.nb * kBN) / 8);
-        store_rows_coalesced<kBN / 8>(
+        const int chunks_ok = min(16, (p.n_out - tile.nb * kBN - 128 * half) / 8);
+        store_rows_coalesced<16>(
             w, reinterpret_cast<uint8_t*>(static_cast<__nv_bfloat16*>(p.out) +
-                                          static_cast<size_t>(row0) * p.n_out + tile.nb * kBN),
+                                          static_cast<size_t>(row0) * p.n_out + tile.nb * kBN +
+                                          128 * half),
             static_cast<size_t>(p.n_out) * 2, rows_ok, chunks_ok, lane);
       }
       ++tiles;
     }
+    pipe.hq = hq;
     pipe.tiles = tiles;
   }
 
