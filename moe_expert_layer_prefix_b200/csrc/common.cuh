@@ -208,20 +208,17 @@ __device__ __forceinline__ void cp_async_4(void* dst_smem, const void* src) {
                : "memory");
 }
 
+// Asynchronous 16-byte global -> shared copy (cached in L2 only).  Both addresses must be
+// 16-byte aligned.
+__device__ __forceinline__ void cp_async_16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src)
+               : "memory");
+}
+
 // One arrival on bar once every cp.async this thread has issued so far has landed; the
 // barrier's expected count must include it (.noinc).
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t* bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
-               : "memory");
-}
-
-// Reads 16 bytes of shared memory and writes them back unchanged, making this thread the
-// generic-proxy writer of bytes another agent (a cp.async) put there.
-__device__ __forceinline__ void smem_touch16(void* p) {
-  uint32_t a, b, c, d;
-  const uint32_t s = smem_u32(p);
-  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(s));
-  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(s), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
 

@@ -60,8 +60,6 @@ namespace gemm {
 constexpr int kBM = 128;           // accumulator rows per CTA (TMEM lanes)
 constexpr int kBN = 256;           // accumulator columns (MMA N)
 constexpr int kRowBytes = 128;     // K bytes per tile row per stage (one swizzle atom)
-constexpr int kSfaBytes = 512;     // 128 rows x 4 UE8M0
-constexpr int kSfbBytes = 1024;    // 256 rows x 4 UE8M0
 constexpr int kTmemCols = 512;
 constexpr int kAccCol = 0;
 constexpr int kSfaCol = 256;       // scale-factor column sets start here ...
@@ -73,8 +71,19 @@ constexpr int kEpiWarps = 8;       // two warps per TMEM lane quadrant, one per 
 constexpr int kThreads = 32 * (4 + kEpiWarps);
 constexpr int kMaxE = 1024;
 constexpr int kMaxStages = 6;
-constexpr int kSfSlots = 16;       // scale-factor ring, decoupled from (and deeper than) the A/B ring
-constexpr int kSfBatch = 8;        // slots the converter publishes with one warp-wide arrive
+// Scale-factor ring: one slot per group of 4 k-steps (16 k-steps ahead of the MMA issuer),
+// decoupled from the A/B ring.  Slot layout (bytes):
+//   [0, 2048)     A: the raw fp32 scales of the CTA's 128 rows, 16 B (4 k-steps) per row,
+//                 rewritten in place into 32 lines x 16 B of UE8M0 (line l, word c = row
+//                 32c + l, byte j = k-step j of the group) -- the 32x128b layout tcgen05.cp reads
+//   [2048, 6144)  B, E2M1: the raw UE8M0 bytes of the tile's 256 rows, 16 B per row (4 k-steps
+//                 x 4 sub-blocks of 32), rewritten in place into 4 k-steps x 2 atoms x 512 B
+//   [2048, 3072)  B, E4M3: 2 atoms x 512 B of UE8M0 (every row of an atom carries the scale
+//                 of its 128-row weight block); the raw fp32 block scales at [3072, 3104)
+constexpr int kSfGroups = 4;
+constexpr int kSfSlotBytes = 6144;
+constexpr int kSfBOff = 2048;
+constexpr int kSfBRawE4 = 3072;
 
 struct TcParams {
   const int32_t* offsets;  // [E+1]
@@ -93,9 +102,9 @@ struct TcParams {
 struct SharedState {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
-  uint64_t sf_raw[kSfSlots];    // loader -> converter: raw scale words staged in the slot
-  uint64_t sf_full[kSfSlots];   // converters -> MMA issuer: slot converted (one per CTA)
-  uint64_t sf_empty[kSfSlots];  // MMA issuer -> loaders: slot copied to TMEM and consumed
+  uint64_t sf_raw[kSfGroups];   // loader -> converter: raw scale words staged in the slot
+  uint64_t sf_full[kSfGroups];  // converters -> MMA issuer: slot converted (one per CTA)
+  uint64_t sf_empty[kSfGroups]; // MMA issuer -> loaders: slot copied to TMEM and consumed
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
@@ -123,7 +132,7 @@ struct Cfg {
   static constexpr int kBTileBytes = kBRows * kRowBytes;  // 32 KB single, 16 KB pair
   static constexpr int kTileM = kTm * kCta;               // rows of one tile
   static constexpr size_t kSmem = 1024 + kStages * (kATileBytes + kBTileBytes) +
-                                  kSfSlots * (kSfaBytes + kSfbBytes) + sizeof(SharedState);
+                                  kSfGroups * kSfSlotBytes + sizeof(SharedState);
   static_assert(kSmem <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
 };
 
@@ -225,7 +234,7 @@ struct Pipe {
   uint32_t prod_it = 0;  // producer: k-steps issued into the ring
   uint32_t mma_it = 0;   // MMA issuer: k-steps consumed
   uint32_t tiles = 0;    // MMA issuer / epilogue: accumulator uses
-  uint32_t sf_it = 0;    // scale loader / converter: k-steps staged
+  uint32_t sf_it = 0;    // scale loader / converter: groups of 4 k-steps staged
   uint32_t sf_grp = 0;   // MMA issuer: groups of 4 k-steps whose scales were copied to TMEM
   uint32_t hq = 0;       // epilogue: linear-1 tiles requantised to E4M3 (amax exchanges)
 };
@@ -245,8 +254,8 @@ __device__ __forceinline__ Smem carve(uint8_t* smem_raw) {
   m.sA = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                     ~static_cast<uintptr_t>(1023));
   m.sB = m.sA + C::kStages * C::kATileBytes;
-  m.sSF = m.sB + C::kStages * C::kBTileBytes;             // per slot: SFA 512 B, SFB 1024 B
-  m.ss = reinterpret_cast<SharedState*>(m.sSF + kSfSlots * (kSfaBytes + kSfbBytes));
+  m.sSF = m.sB + C::kStages * C::kBTileBytes;             // kSfGroups slots of kSfSlotBytes
+  m.ss = reinterpret_cast<SharedState*>(m.sSF + kSfGroups * kSfSlotBytes);
   return m;
 }
 
@@ -261,7 +270,7 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
       mbar_init(&ss.full[s], 1);
       mbar_init(&ss.empty[s], 1);
     }
-    for (int s = 0; s < kSfSlots; ++s) {
+    for (int s = 0; s < kSfGroups; ++s) {
       mbar_init(&ss.sf_raw[s], 32);  // one cp.async completion arrival per loader lane
       mbar_init(&ss.sf_full[s], kCta);
       mbar_init(&ss.sf_empty[s], 1);
@@ -427,14 +436,15 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
             ok = false;
             break;
           }
-          const int slot = static_cast<int>(it % kSfSlots);
           const bool grp_start = (kb & 3) == 0;
+          const bool grp_end = (kb & 3) == 3 || kb == KB - 1;
+          // this k-step's group: grp counts the groups started so far (this one included
+          // once its first k-step has passed)
+          const uint32_t gcur = grp_start ? grp : grp - 1u;
+          const int slot = static_cast<int>(gcur % kSfGroups);
           if constexpr (kBlockScaled) {
-            // the scales of a group of 4 k-steps are published together; slots are converted
-            // and published in order, so the group's last slot covers the whole group
             if (grp_start) {
-              const uint32_t il = it + static_cast<uint32_t>(min(kb + 3, KB - 1) - kb);
-              if (!mbar_wait<kPair>(&ss.sf_full[il % kSfSlots], (il / kSfSlots) & 1u, p.err,
+              if (!mbar_wait<kPair>(&ss.sf_full[slot], (gcur / kSfGroups) & 1u, p.err,
                                     SITE_GEMM_FULL, abort)) {
                 ok = false;
                 break;
@@ -452,18 +462,20 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           const uint32_t tsfb =
               tmem + kSfbCol + (kBFmt == 5 ? it % kSfSets : grp % kSfSets) * kSfSetCols;
           if constexpr (kBlockScaled) {
-            const uint32_t sf = smem_u32(sSF + slot * (kSfaBytes + kSfbBytes));
+            const uint32_t sf = smem_u32(sSF + slot * kSfSlotBytes);
             if (grp_start) {
               if constexpr (kPair) tc_cp_32x128b_warpx4_pair(tsfa, desc_sf_32x16(sf));
               else tc_cp_32x128b_warpx4(tsfa, desc_sf_32x16(sf));
             }
             if (kBFmt == 5 || grp_start) {
+              // E2M1: this k-step's 2 atoms; E4M3: the group's 2 atoms
+              const uint32_t sfb = sf + kSfBOff + (kBFmt == 5 ? 1024u * static_cast<uint32_t>(kb & 3) : 0u);
               if constexpr (kPair) {
-                tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sf + kSfaBytes));
-                tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+                tc_cp_32x128b_warpx4_pair(tsfb, desc_sf_32x16(sfb));
+                tc_cp_32x128b_warpx4_pair(tsfb + 4, desc_sf_32x16(sfb + 512));
               } else {
-                tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sf + kSfaBytes));
-                tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sf + kSfaBytes + 512));
+                tc_cp_32x128b_warpx4(tsfb, desc_sf_32x16(sfb));
+                tc_cp_32x128b_warpx4(tsfb + 4, desc_sf_32x16(sfb + 512));
               }
             }
           }
@@ -490,8 +502,10 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           if constexpr (kPair) tc_commit_pair(&ss.empty[stage], 0x3);
           else tc_commit(&ss.empty[stage]);
           if constexpr (kBlockScaled) {
-            if constexpr (kPair) tc_commit_pair(&ss.sf_empty[slot], 0x3);
-            else tc_commit(&ss.sf_empty[slot]);
+            if (grp_end) {  // the group's slot is free once its last k-step's MMAs are done
+              if constexpr (kPair) tc_commit_pair(&ss.sf_empty[slot], 0x3);
+              else tc_commit(&ss.sf_empty[slot]);
+            }
           }
           ++it;
         }
@@ -516,21 +530,27 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     }
   } else if (warp == 2) {
     // ------------------------------------------------------------------ scale loader
-    // Iterations i = (tile, k-step) of this CTA in order; iteration i uses scale slot
-    // i % kSfSlots.  Each lane copies the raw scale words of its rows straight into the slot
-    // at their final positions with asynchronous 4-byte copies whose completion arrives on the
-    // slot's raw barrier, so the loader runs up to kSfSlots k-steps ahead of the MMA issuer
-    // with nothing held in registers; row pointers are set up once per tile.  Each CTA copies
-    // the scales of its own A rows and of all 256 B rows of the tile; the converter warp then
-    // rewrites the slot in place.
+    // Groups g = (tile, 4 consecutive k-steps) of this CTA in order; group g uses scale slot
+    // g % kSfGroups.  Each lane copies the raw scales of its rows straight into the slot with
+    // asynchronous copies (one 16-byte copy per row and group where the rows are 16-byte
+    // aligned and the group is whole, else one 4-byte copy per k-step) whose completion
+    // arrives on the slot's raw barrier, so the loader runs up to kSfGroups groups ahead of
+    // the MMA issuer with nothing held in registers; row pointers are set up once per tile.
+    // Each CTA copies the scales of its own 128 A rows and those the tile's B rows need; the
+    // converter warp then rewrites the slot in place.
     if constexpr (kBlockScaled) {
-      constexpr int kNB = kBFmt == 5 ? 8 : 2;  // B words per lane per k-step
+      constexpr int kNB = kBFmt == 5 ? 8 : 2;  // B rows (E2M1) or weight blocks (E4M3) per lane
       const int KS = p.K / 128;                // fp32 scale columns of A (and of E4M3 B)
+      const int NG = (KB + 3) / 4;             // groups per tile
+      // 16-byte copies need the base pointer and every row start 16-byte aligned
+      const bool a16 = (KS % 4) == 0 && (reinterpret_cast<uintptr_t>(p.a_scales) & 15u) == 0;
+      const bool b16 = (kBFmt == 5 ? ((p.K / 32) % 16) == 0 : (KS % 4) == 0) &&
+                       (reinterpret_cast<uintptr_t>(p.b_scales) & 15u) == 0;
       const float* pa[4];
       const uint8_t* pb[kNB];
       const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
-      const uint32_t it0 = pipe.sf_it;
-      uint32_t gi = it0;
+      const uint32_t g0 = pipe.sf_it;
+      uint32_t gi = g0;
       bool ok = true;
       for (int lt = cid; lt < total && ok; lt += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
@@ -543,14 +563,15 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
         const int wr0 = kSwiGLU ? tile.nb * 128 : tile.nb * kBN;     // first B row, atom 0
         const int wr1 = kSwiGLU ? p.I + tile.nb * 128 : wr0 + 128;   // first B row, atom 1
         if constexpr (kBFmt == 5) {
+          // lane l stages rows 128a + 32c + l of the tile (a = atom, c = 0..3)
 #pragma unroll
           for (int a = 0; a < 2; ++a)
 #pragma unroll
-            for (int r1 = 0; r1 < 4; ++r1) {
-              int wr = (a == 0 ? wr0 : wr1) + lane + 32 * r1;
+            for (int c = 0; c < 4; ++c) {
+              int wr = (a == 0 ? wr0 : wr1) + lane + 32 * c;
               wr = wr < p.w_rows ? wr : p.w_rows - 1;
-              pb[a * 4 + r1] = static_cast<const uint8_t*>(p.b_scales) +
-                               (static_cast<size_t>(tile.e) * p.w_rows + wr) * (p.K / 32);
+              pb[a * 4 + c] = static_cast<const uint8_t*>(p.b_scales) +
+                              (static_cast<size_t>(tile.e) * p.w_rows + wr) * (p.K / 32);
             }
         } else {
 #pragma unroll
@@ -562,109 +583,138 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
                 (static_cast<size_t>(tile.e) * (p.w_rows / 128) + wr / 128) * KS);
           }
         }
-        for (int kb = 0; kb < KB; ++kb, ++gi) {
-          const int slot = static_cast<int>(gi % kSfSlots);
-          if (!mbar_wait<kPair>(&ss.sf_empty[slot], ((gi / kSfSlots) & 1u) ^ 1u, p.err,
+        for (int g = 0; g < NG; ++g, ++gi) {
+          const int slot = static_cast<int>(gi % kSfGroups);
+          if (!mbar_wait<kPair>(&ss.sf_empty[slot], ((gi / kSfGroups) & 1u) ^ 1u, p.err,
                                 SITE_GEMM_SF_EMPTY, abort)) {
             ok = false;
             break;
           }
-          uint8_t* sf = sSF + slot * (kSfaBytes + kSfbBytes);
+          uint8_t* sf = sSF + slot * kSfSlotBytes;
+          const int nk = min(4, KB - 4 * g);  // k-steps in this group
+          const bool whole = nk == 4;
 #pragma unroll
-          for (int r1 = 0; r1 < 4; ++r1) cp_async_4(sf + 16 * lane + 4 * r1, pa[r1] + kb);
+          for (int r1 = 0; r1 < 4; ++r1) {
+            uint8_t* dst = sf + 16 * (lane + 32 * r1);
+            const float* src = pa[r1] + 4 * g;
+            if (a16 && whole) {
+              cp_async_16(dst, src);
+            } else {
+              for (int j = 0; j < nk; ++j) cp_async_4(dst + 4 * j, src + j);
+            }
+          }
           if constexpr (kBFmt == 5) {
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
-              cp_async_4(sf + kSfaBytes + 512 * (r >> 2) + 16 * lane + 4 * (r & 3), pb[r] + 4 * kb);
-          } else {
-#pragma unroll
-            for (int a = 0; a < 2; ++a)
-              cp_async_4(sf + kSfaBytes + 16 * lane + 4 * a,
-                         reinterpret_cast<const float*>(pb[a]) + kb);
+            for (int r = 0; r < 8; ++r) {
+              uint8_t* dst = sf + kSfBOff + 16 * (128 * (r >> 2) + 32 * (r & 3) + lane);
+              const uint8_t* src = pb[r] + 16 * g;
+              if (b16 && whole) {
+                cp_async_16(dst, src);
+              } else {
+                for (int j = 0; j < nk; ++j) cp_async_4(dst + 4 * j, src + 4 * j);
+              }
+            }
+          } else if (lane < 2) {
+            uint8_t* dst = sf + kSfBRawE4 + 16 * lane;
+            const float* src = reinterpret_cast<const float*>(pb[lane]) + 4 * g;
+            if (b16 && whole) {
+              cp_async_16(dst, src);
+            } else {
+              for (int j = 0; j < nk; ++j) cp_async_4(dst + 4 * j, src + j);
+            }
           }
           cp_async_mbar_arrive(&ss.sf_raw[slot]);
         }
       }
       cp_async_wait_all();  // no copy may still be landing when the CTA moves on
-      pipe.sf_it = it0 + static_cast<uint32_t>(my_tiles * KB);
+      pipe.sf_it = g0 + static_cast<uint32_t>(my_tiles * NG);
     }
   } else if (warp == 3) {
     // ------------------------------------------------------------------ scale converter
-    // Rewrites the staged raw words into the layout tcgen05.cp reads: per 128-row atom, 32
-    // lines of 16 bytes, byte 16*(r%32) + 4*(r/32) + b for row r, one UE8M0 (the exponent
-    // byte of a power-of-two fp32 scale) per byte.  A scales and E4M3 B scales cover 128 of K,
-    // so b indexes the k-step inside a group of 4 k-steps of a tile: once the group's last
-    // k-step is staged, its packed atoms are written into the slot of the group's first
-    // k-step (one TMEM copy per group).  E2M1 B scales are per 32 of K and already UE8M0 in
-    // atom order (b = sub-block).  kSfBatch slots are published at a time with one warp-wide
-    // arrive on the (pair leader's) slot barriers, so the cluster-scope release that makes
-    // them visible is paid once per batch; kSfBatch + 4 <= kSfSlots keeps the loader free to
-    // stage every slot a published group needs.  A scale word that is not a positive normal
+    // Rewrites each staged group in place into the layout tcgen05.cp reads: per 128-row
+    // atom, 32 lines of 16 bytes, line l word c for row 32c + l, one UE8M0 per byte.  A and
+    // E4M3 B scales cover 128 of K, so byte j of a word is k-step j of the group (one TMEM
+    // copy per group; the MMA's scale-byte selector picks the k-step); the UE8M0 byte of a
+    // power-of-two fp32 scale is its exponent field.  E2M1 B scales are per 32 of K and
+    // already UE8M0: each k-step gets its own 2 atoms (byte = sub-block).  Lane l reads only
+    // rows congruent to l mod 32 and writes only lines that held such rows, so the in-place
+    // rewrite needs no exchange between lanes.  A scale word that is not a positive normal
     // power of two (no exact UE8M0 byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
-    static_assert(kSfBatch + 4 <= kSfSlots, "scale ring too shallow for batch + group");
     if constexpr (kBlockScaled) {
+      const int NG = (KB + 3) / 4;
       const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
-      const int n_iter = my_tiles * KB;
-      const uint32_t it0 = pipe.sf_it;
+      const int n_grp = my_tiles * NG;
+      const uint32_t g0 = pipe.sf_it;
       const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
-      bool ok = true;
       uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
-      for (int b = 0; b < n_iter && ok; b += kSfBatch) {
-        const int cnt = n_iter - b < kSfBatch ? n_iter - b : kSfBatch;
-        for (int j = 0; j < cnt; ++j) {
-          const uint32_t gi = it0 + static_cast<uint32_t>(b + j);
-          const int slot = static_cast<int>(gi % kSfSlots);
-          if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfSlots) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sf = sSF + slot * (kSfaBytes + kSfbBytes);
-          if constexpr (kBFmt == 5) {
-            // rewritten so that this warp's proxy fence covers every byte tcgen05.cp reads
-            smem_touch16(sf + kSfaBytes + 16 * lane);
-            smem_touch16(sf + kSfaBytes + 512 + 16 * lane);
-          }
-          const int kb = (b + j) % KB;
-          const int g0 = kb & ~3;
-          if (kb == KB - 1 || (kb & 3) == 3) {
-            uint32_t wa0 = 0, wa1 = 0, wa2 = 0, wa3 = 0, wb0 = 0, wb1 = 0;
-            for (int q = 0; q <= kb - g0; ++q) {
-              const uint8_t* src =
-                  sSF + ((gi - static_cast<uint32_t>(kb - g0 - q)) % kSfSlots) * (kSfaBytes + kSfbBytes);
-              const uint4 a = *reinterpret_cast<const uint4*>(src + 16 * lane);
-              wa0 |= ((a.x >> 23) & 0xFFu) << (8 * q);
-              wa1 |= ((a.y >> 23) & 0xFFu) << (8 * q);
-              wa2 |= ((a.z >> 23) & 0xFFu) << (8 * q);
-              wa3 |= ((a.w >> 23) & 0xFFu) << (8 * q);
-              bad |= not_pow2_scale(a.x) | not_pow2_scale(a.y) | not_pow2_scale(a.z) |
-                     not_pow2_scale(a.w);
-              if constexpr (kBFmt != 5) {
-                const uint2 w2 = *reinterpret_cast<const uint2*>(src + kSfaBytes + 16 * lane);
-                wb0 |= ((w2.x >> 23) & 0xFFu) << (8 * q);
-                wb1 |= ((w2.y >> 23) & 0xFFu) << (8 * q);
-                bad |= not_pow2_scale(w2.x) | not_pow2_scale(w2.y);
-              }
-            }
-            uint8_t* dst =
-                sSF + ((gi - static_cast<uint32_t>(kb - g0)) % kSfSlots) * (kSfaBytes + kSfbBytes);
-            *reinterpret_cast<uint4*>(dst + 16 * lane) = make_uint4(wa0, wa1, wa2, wa3);
-            if constexpr (kBFmt != 5) {
-              *reinterpret_cast<uint4*>(dst + kSfaBytes + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
-              *reinterpret_cast<uint4*>(dst + kSfaBytes + 512 + 16 * lane) =
-                  make_uint4(wb1, wb1, wb1, wb1);
+      for (int i = 0; i < n_grp; ++i) {
+        const uint32_t gi = g0 + static_cast<uint32_t>(i);
+        const int slot = static_cast<int>(gi % kSfGroups);
+        if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfGroups) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort))
+          break;
+        uint8_t* sf = sSF + slot * kSfSlotBytes;
+        const int nk = min(4, KB - 4 * (i % NG));
+        // A: rows lane + 32c -> line lane
+        uint32_t wa[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sf + 16 * (lane + 32 * c));
+          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+          uint32_t w = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              w |= ((x[j] >> 23) & 0xFFu) << (8 * j);
+              bad |= not_pow2_scale(x[j]);
             }
           }
+          wa[c] = w;
         }
-        if (!ok) break;
+        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        if constexpr (kBFmt == 5) {
+          // rows 128a + 32c + lane, 16 B each (k-step j = word j) -> line (k-step j, atom a)
+          uint4 v[2][4];
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              v[a][c] = *reinterpret_cast<const uint4*>(sf + kSfBOff + 16 * (128 * a + 32 * c + lane));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              const uint32_t w0 = j == 0 ? v[a][0].x : j == 1 ? v[a][0].y : j == 2 ? v[a][0].z : v[a][0].w;
+              const uint32_t w1 = j == 0 ? v[a][1].x : j == 1 ? v[a][1].y : j == 2 ? v[a][1].z : v[a][1].w;
+              const uint32_t w2 = j == 0 ? v[a][2].x : j == 1 ? v[a][2].y : j == 2 ? v[a][2].z : v[a][2].w;
+              const uint32_t w3 = j == 0 ? v[a][3].x : j == 1 ? v[a][3].y : j == 2 ? v[a][3].z : v[a][3].w;
+              *reinterpret_cast<uint4*>(sf + kSfBOff + 1024 * j + 512 * a + 16 * lane) =
+                  make_uint4(w0, w1, w2, w3);
+            }
+        } else {
+          // the two weight blocks' scales, the same for every row of their atom
+          const uint4 rg = *reinterpret_cast<const uint4*>(sf + kSfBRawE4);
+          const uint4 ru = *reinterpret_cast<const uint4*>(sf + kSfBRawE4 + 16);
+          const uint32_t xg[4] = {rg.x, rg.y, rg.z, rg.w}, xu[4] = {ru.x, ru.y, ru.z, ru.w};
+          uint32_t wb0 = 0, wb1 = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              wb0 |= ((xg[j] >> 23) & 0xFFu) << (8 * j);
+              wb1 |= ((xu[j] >> 23) & 0xFFu) << (8 * j);
+              bad |= not_pow2_scale(xg[j]) | not_pow2_scale(xu[j]);
+            }
+          }
+          *reinterpret_cast<uint4*>(sf + kSfBOff + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
+          *reinterpret_cast<uint4*>(sf + kSfBOff + 512 + 16 * lane) = make_uint4(wb1, wb1, wb1, wb1);
+        }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane < cnt) {
-          const int slot = static_cast<int>((it0 + static_cast<uint32_t>(b + lane)) % kSfSlots);
+        if (lane == 0) {
           if constexpr (kPair) mbar_arrive_cluster(full_lead0 + slot * sizeof(uint64_t));
           else mbar_arrive(&ss.sf_full[slot]);
         }
       }
-      pipe.sf_it = it0 + n_iter;
+      pipe.sf_it = g0 + static_cast<uint32_t>(n_grp);
       // the exponent fields were used all the same: the result is undefined, the call fails
       if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
     }
