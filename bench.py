@@ -183,7 +183,16 @@ def run_native(args, ws, rank, local):
             raise SystemExit("--bf16-input needs a workload with E4M3 activations")
         d["x"] = synth.make_activations(dataclasses.replace(wl, act="bf16"), dev)["x"]
         d["x_scales"] = None
-    W = M.Weights(wl.act, wl.wt, d["w1"], d["w2"], d["w1_scales"], d["w2_scales"])
+    if args.scale_fmt == "fp32":
+        # arbitrary fp32 block scales: the power-of-two scales times seeded factors in
+        # [1.05, 1.95] (no scale stays a power of two)
+        if wl.act != "e4m3" or wl.wt != "e4m3":
+            raise SystemExit("--scale-fmt fp32 needs E4M3 activations and weights")
+        g = torch.Generator(device=dev).manual_seed(1234)
+        for n in ("x_scales", "w1_scales", "w2_scales"):
+            d[n] = (d[n] * (1.05 + 0.9 * torch.rand(d[n].shape, generator=g, device=dev))).contiguous()
+    W = M.Weights(wl.act, wl.wt, d["w1"], d["w2"], d["w1_scales"], d["w2_scales"],
+                  scale_fmt=args.scale_fmt)
     T, H, E, k, I, S = wl.T, wl.H, wl.E, wl.k, wl.I, wl.S
     stream = torch.cuda.current_stream()
 
@@ -400,7 +409,9 @@ def run_native(args, ws, rank, local):
                    "l2": "inputs larger than L2 (expert weights >> 126 MB), no flush",
                    "parallelism": f"replicas x{ws}"},
         "tflops": wl.flops() / (ms / 1e3) / 1e12 * ws,
-        "step": "moe_forward (one persistent launch per step)",
+        "step": ("moe_forward (one persistent launch per step)" if args.scale_fmt == "pow2"
+                 else "moe_forward (fp32 block scales: the chain of entry points, 9 launches)"),
+        "scale_fmt": args.scale_fmt,
         "chain_ms_per_step": chain_ms,
         "stage_ms": stage_ms,
         "roofline": roof,
@@ -417,6 +428,78 @@ def run_native(args, ws, rank, local):
     if ws == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, d, args.cpu_tokens)
     return res
+
+
+def run_backward(args, ws, rank, local):
+    """The BF16 layer's backward (moe_expert_backward: combine and router backward, the
+    recomputed pre-activations, dh, SwiGLU backward, dx and both weight gradients) from the
+    forward's stored tensors, timed per call with CUDA events."""
+    import moe_expert_layer_prefix_b200 as M
+
+    wl = workload(args)
+    if wl.act != "bf16" or wl.wt != "bf16":
+        raise SystemExit("--backward runs the BF16 layer (e.g. --workload mixtral_bf16)")
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = synth.make_inputs(wl, dev)
+    W = M.Weights(wl.act, wl.wt, d["w1"], d["w2"], d["w1_scales"], d["w2_scales"])
+    T, H, E, k, I, S = wl.T, wl.H, wl.E, wl.k, wl.I, wl.S
+    idx, gw = M.moe_route(d["logits"], k, wl.score, bias=d["bias"], renorm=wl.renorm)
+    r = M.moe_dispatch(d["x"], idx, E, wl.act)
+    h, _ = M.moe_expert_linear1(r["x_perm"], r["expert_offsets"], W)
+    y = M.moe_expert_linear2(h, r["expert_offsets"], W)
+    w1_t, w2_t = M.moe_transpose_experts(W.w1), M.moe_transpose_experts(W.w2)
+    g = torch.Generator(device=dev).manual_seed(99)
+    dout = (torch.randn((T, H), generator=g, device=dev) / 64).to(torch.bfloat16)
+    bws = M.workspace(M.moe_workspace_size("backward", T, H, E, k, I, "bf16", "bf16"), dev)
+
+    def step():
+        return M.moe_expert_backward(dout, d["logits"], idx, gw, r["expert_offsets"], r["slot_of"],
+                                     r["x_perm"], h, y, W, w1_t, w2_t, k, score=wl.score,
+                                     renorm=wl.renorm, ws=bws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, site = M.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {M.moe_status_string(st)} at site {site}")
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    stream = torch.cuda.current_stream()
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    n0 = M.moe_launch_count()
+    for i in range(args.steps):
+        evs[i].record(stream)
+        step()
+    evs[-1].record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    launches = M.moe_launch_count() - n0
+    clk = clocks.stop()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+    ms = max_over_ranks(float(np.sum(per)), ws) / args.steps
+    # algorithmic FLOPs of the backward's GEMMs per step: G recomputed 4SHI, dh 2SHI,
+    # dx_slot 4SHI, dW1 4SHI, dW2 2SHI
+    flops = 16.0 * S * H * I
+    pk, pk_kind = peaks()
+    ach = flops / (ms / 1e3) / 1e12
+    roof = {"bound": "tensor", "achieved": ach, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": ach / pk["bf16_tflops"], "traffic": None, "kernel": "moe_expert_backward (whole call)",
+            "peak_note": f"{pk_kind} bf16 burst; the call's five GEMMs against the whole call's time"}
+    return {
+        "metric": "MoE layer backward tokens/s (1 B200 per replica)",
+        "value": T * ws / (ms / 1e3), "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "T": T, "H": H, "E": E, "k": k, "I": I,
+                   "l2": "inputs larger than L2 (weights >> 126 MB), no flush",
+                   "parallelism": f"replicas x{ws}"},
+        "tflops": ach, "step": "moe_expert_backward", "roofline": roof,
+        "gpu_launches": int(launches), "clocks": clk,
+    }
 
 
 def _oracle_layer(wl, d):
@@ -500,6 +583,11 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--bf16-input", action="store_true",
                     help="E4M3 workloads: feed BF16 activations, quantised in the dispatch")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the BF16 layer's backward (moe_expert_backward) instead")
+    ap.add_argument("--scale-fmt", default="pow2", choices=["pow2", "fp32"],
+                    help="E4M3 layers: power-of-two block scales (UE8M0 tensor-core path) or "
+                         "arbitrary fp32 block scales (per-block promotion)")
     ap.add_argument("--tiles", default="auto", choices=["auto", "single", "pair", "small"],
                     help="tile shape of the expert GEMMs")
     ap.add_argument("--T", type=int, default=None, help="override T (profiling captures)")
@@ -515,6 +603,8 @@ def main():
     ws, rank, local = dist_setup(args)
     if args.impl == "reference":
         res = run_reference(args, ws, rank) if rank == 0 else None
+    elif args.backward:
+        res = run_backward(args, ws, rank, local)
     else:
         res = run_native(args, ws, rank, local)
     if rank == 0 and res is not None:

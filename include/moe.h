@@ -76,6 +76,17 @@ typedef enum moe_op {
  * projection.  W2 [E, H, I].  Both K-major (each output row contiguous over the reduction
  * dimension).  Scales: E4M3 -> fp32 [E, 2I/128, H/128] and [E, H/128, I/128];
  * E2M1 -> UE8M0 bytes [E, 2I, H/32] and [E, H, I/32]; F32 / BF16 -> NULL. */
+/* What the fp32 block scales of an E4M3 layer hold (activation scales x_scales /
+ * x_perm_scales and the E4M3 weight scales alike).
+ *   MOE_SCALE_POW2  positive normal powers of two: they convert exactly to the UE8M0 scales
+ *                   the block-scaled tensor-core MMA applies (the fast path; any other value
+ *                   is reported on the device as MOE_ERR_UNSUPPORTED at site 301)
+ *   MOE_SCALE_FP32  any positive finite fp32 values: the expert GEMMs run unscaled E4M3
+ *                   MMAs per 128-deep block of K and fold each block's partial sum into an
+ *                   fp32 accumulator with its scales (E4M3 weights only; the layer runs as
+ *                   the chain of entry points, also under moe_forward) */
+typedef enum moe_scale_fmt { MOE_SCALE_POW2 = 0, MOE_SCALE_FP32 = 1 } moe_scale_fmt;
+
 typedef struct moe_weights {
   int act; /* moe_dtype of x, x_perm and h */
   int wt;  /* moe_dtype of W1 and W2 */
@@ -83,6 +94,7 @@ typedef struct moe_weights {
   const void* w1_scales;
   const void* w2;
   const void* w2_scales;
+  int scale_fmt; /* moe_scale_fmt (0, the power-of-two scales, when zero-initialised) */
 } moe_weights;
 
 /* Router: per token, select k experts and their gate weights.
@@ -276,7 +288,9 @@ typedef struct moe_backward_args {
  *   dh = BF16(dy_w W2)       (expert GEMM on W2^T)
  *   dG = BF16(SwiGLU backward of G, dh)
  *   dx_slot = BF16(dG W1)    (expert GEMM on W1^T);  dx[t] = BF16(sum of its k slots)
- *   dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e  (fp32)
+ *   dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e  (fp32; tensor cores, on copies of the
+ *                                               operands transposed so that each expert's
+ *                                               slots form a zero-padded 64-column segment)
  * BF16 layers only (the arguments carry no formats).  BF16 tensors, dw1 and dw2 must be
  * 16-byte aligned, the other arrays 4-byte aligned.  Workspace:
  * moe_workspace_size(MOE_OP_BACKWARD, T, H, E, k, I, MOE_BF16, MOE_BF16) bytes, 256-byte

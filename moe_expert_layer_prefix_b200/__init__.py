@@ -55,7 +55,10 @@ class MoeBackwardArgs(ctypes.Structure):
 
 class MoeWeights(ctypes.Structure):
     _fields_ = [("act", ctypes.c_int), ("wt", ctypes.c_int), ("w1", _P), ("w1_scales", _P),
-                ("w2", _P), ("w2_scales", _P)]
+                ("w2", _P), ("w2_scales", _P), ("scale_fmt", ctypes.c_int)]
+
+
+SCALE_FMTS = {"pow2": 0, "fp32": 1}
 
 
 def _sig(name, res, args):
@@ -172,15 +175,19 @@ def workspace(nbytes: int, device) -> torch.Tensor:
 class Weights:
     """Expert weights in the library's layout (see include/moe.h); holds the tensors alive."""
 
-    def __init__(self, act, wt, w1, w2, w1_scales=None, w2_scales=None):
+    def __init__(self, act, wt, w1, w2, w1_scales=None, w2_scales=None, scale_fmt="pow2"):
+        """scale_fmt: 'pow2' (fp32 block scales that are powers of two: the UE8M0 fast path)
+        or 'fp32' (any positive finite fp32 scales; E4M3 weights only)."""
         self.act, self.wt = act, wt
         self.w1, self.w2, self.w1_scales, self.w2_scales = w1, w2, w1_scales, w2_scales
+        self.scale_fmt = scale_fmt
         self.E = w1.shape[0]
         self.H = w1.shape[2] * (2 if wt == "e2m1" else 1)
         self.I = w2.shape[2] * (2 if wt == "e2m1" else 1)
         self.c = MoeWeights(DTYPES[act], DTYPES[wt], w1.data_ptr(),
                             None if w1_scales is None else w1_scales.data_ptr(), w2.data_ptr(),
-                            None if w2_scales is None else w2_scales.data_ptr())
+                            None if w2_scales is None else w2_scales.data_ptr(),
+                            SCALE_FMTS[scale_fmt])
 
 
 def _groups(groups):

@@ -100,6 +100,9 @@ moe_status check_weights(const moe_weights* W, int need_act) {
     return MOE_ERR_INVALID_ARG;
   if (need_act >= 0 && W->act != need_act) return MOE_ERR_INVALID_ARG;
   if (!valid_pair(W->act, W->wt)) return MOE_ERR_UNSUPPORTED;
+  if (W->scale_fmt != MOE_SCALE_POW2 && W->scale_fmt != MOE_SCALE_FP32) return MOE_ERR_INVALID_ARG;
+  if (W->scale_fmt == MOE_SCALE_FP32 && (W->act != MOE_E4M3 || W->wt != MOE_E4M3))
+    return MOE_ERR_UNSUPPORTED;
   const bool scaled = W->wt == MOE_E4M3 || W->wt == MOE_E2M1;
   if (scaled && (W->w1_scales == nullptr || W->w2_scales == nullptr)) return MOE_ERR_INVALID_ARG;
   const size_t a = W->wt == MOE_E2M1 ? 32 : 16;
@@ -177,6 +180,10 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       b += round256(static_cast<size_t>(S) * 2 * I * 2) * 2;  // G, dG
       b += round256(static_cast<size_t>(S) * I * 2);          // dh
       b += round256(static_cast<size_t>(S) * 4) * 2;          // dgates, unit weights
+      b += round256(static_cast<size_t>(E + 1) * 4);          // padded segment starts
+      // the transposed, expert-padded operands of one weight gradient at a time
+      b += round256(static_cast<size_t>(2 * I + H > H + I ? 2 * I + H : H + I) *
+                    wgrad_pad_cols(S, E) * 2);
       return b;
     }
     case MOE_OP_FORWARD: {
@@ -191,6 +198,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       b += h_bytes(S, I, act);
       b += round256(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));  // y
       b += 256;                                                               // grid barrier
+      b += round256(static_cast<size_t>(forward_mb_cap(S, E)) * 2 * 4);       // tile counters
       return b;
     }
     default:
@@ -309,7 +317,7 @@ moe_status moe_expert_linear1(const void* x_perm, const float* x_perm_scales,
   if (st != MOE_OK) return st;
   if (W->act == MOE_E4M3 && !h_scales) return MOE_ERR_INVALID_ARG;
   FfnArgs a{W->act, W->wt, x_perm, x_perm_scales, expert_offsets, S, H, I, E,
-            W->w1, W->w1_scales, h, h_scales, device_error_word()};
+            W->w1, W->w1_scales, h, h_scales, device_error_word(), W->scale_fmt};
   return run_ffn(1, a, stream);
 }
 
@@ -321,7 +329,7 @@ moe_status moe_expert_linear2(const void* h, const float* h_scales, const int32_
   moe_status st = check_ffn(h, h_scales, expert_offsets, S, H, I, E, W, y);
   if (st != MOE_OK) return st;
   FfnArgs a{W->act, W->wt, h, h_scales, expert_offsets, S, H, I, E,
-            W->w2, W->w2_scales, y, nullptr, device_error_word()};
+            W->w2, W->w2_scales, y, nullptr, device_error_word(), W->scale_fmt};
   return run_ffn(2, a, stream);
 }
 
@@ -406,12 +414,14 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
   void* ffn_ws = take(h_bytes(S, I, act));
   void* y = take(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));
   uint32_t* bar = reinterpret_cast<uint32_t*>(take(256));
+  uint32_t* counters =
+      reinterpret_cast<uint32_t*>(take(static_cast<size_t>(forward_mb_cap(S, E)) * 2 * 4));
   if (topk_idx_out) topk_idx = topk_idx_out;
   if (topk_w_out) topk_w = topk_w_out;
   if (offsets_out) offsets = offsets_out;
 
-  if (act != MOE_F32) {
-    // tensor-core formats: the whole layer in one persistent launch
+  if (act != MOE_F32 && W->scale_fmt == MOE_SCALE_POW2) {
+    // tensor-core formats with power-of-two scales: the whole layer in one persistent launch
     if (!aligned(logits, 4) || (bias && !aligned(bias, 4)) || !aligned(out, 16) ||
         !aligned(x, 16) || (x_scales && !aligned(x_scales, 4)))
       return MOE_ERR_MISALIGNED;
@@ -453,6 +463,7 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
     fa.y = y;
     fa.out = out;
     fa.bar = bar;
+    fa.counters = counters;
     fa.err = device_error_word();
     return cuda_status(launch_forward_fused(fa, stream));
   }
@@ -526,6 +537,9 @@ moe_status moe_expert_backward(const moe_backward_args* a, void* ws, size_t ws_b
   void* dh = take(static_cast<size_t>(S) * I * 2);
   float* dgates = static_cast<float*>(take(static_cast<size_t>(S) * 4));
   float* ones = static_cast<float*>(take(static_cast<size_t>(S) * 4));
+  int32_t* pk = static_cast<int32_t*>(take(static_cast<size_t>(E + 1) * 4));
+  const size_t Kp = wgrad_pad_cols(S, E);
+  char* tbuf = static_cast<char*>(take(static_cast<size_t>(2 * I + H > H + I ? 2 * I + H : H + I) * Kp * 2));
   int* err = device_error_word();
   // combine and router backward
   if (launch_combine_backward(a->dout, a->y, a->slot_of, a->topk_w, T, k, H, dy_w, dgates,
@@ -553,11 +567,20 @@ moe_status moe_expert_backward(const moe_backward_args* a, void* ws, size_t ws_b
   if (launch_combine(dx_slot, 0, a->slot_of, ones, T, k, H, a->dx, 0, stream) !=
       cudaSuccess)
     return MOE_ERR_CUDA;
-  // weight gradients
-  if (launch_wgrad(dG, a->x_perm, a->expert_offsets, E, 2 * I, H, a->dw1, stream) !=
-      cudaSuccess)
+  // weight gradients on tensor cores: both operands transposed into expert-padded copies
+  // (dG^T [2I, Kp] and x^T [H, Kp], then dy_w^T [H, Kp] and h^T [I, Kp], one pair at a time)
+  const int32_t* offs = a->expert_offsets;
+  void* at = tbuf;
+  if (launch_wgrad_pad_offsets(offs, E, pk, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  void* bt = tbuf + static_cast<size_t>(2 * I) * Kp * 2;
+  if (launch_pad_transpose(dG, S, 2 * I, offs, pk, E, at, stream) != cudaSuccess ||
+      launch_pad_transpose(a->x_perm, S, H, offs, pk, E, bt, stream) != cudaSuccess ||
+      launch_wgrad_tc(at, bt, offs, pk, S, E, 2 * I, H, a->dw1, err, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (launch_wgrad(dy_w, a->h, a->expert_offsets, E, H, I, a->dw2, stream) != cudaSuccess)
+  bt = tbuf + static_cast<size_t>(H) * Kp * 2;
+  if (launch_pad_transpose(dy_w, S, H, offs, pk, E, at, stream) != cudaSuccess ||
+      launch_pad_transpose(a->h, S, I, offs, pk, E, bt, stream) != cudaSuccess ||
+      launch_wgrad_tc(at, bt, offs, pk, S, E, H, I, a->dw2, err, stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;
 }

@@ -12,7 +12,8 @@
 //   weights:  dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e  (sums over the expert's slots)
 // The activation gradients (dh = dy_w W2, dx_slot = dG W1) and the recomputed
 // pre-activations (G = x W1^T) run on the forward pass's tensor-core expert GEMM, given the
-// weights in the layout it reads (transpose_kernel below makes the transposed copies).
+// weights in the layout it reads (transpose_kernel below makes the transposed copies); the
+// weight gradients run on tensor cores in wgrad_tc.cu.
 #include "common.cuh"
 #include "internal.h"
 
@@ -182,53 +183,6 @@ __global__ void __launch_bounds__(256) swiglu_backward_kernel(const __nv_bfloat1
   }
 }
 
-// Weight gradient out[e] [M, N] (fp32) = A_e^T B_e, A [S, M] and B [S, N] BF16, e's rows
-// offsets[e] .. offsets[e+1]: a 64 x 64 output tile per block, 16 rows of A and B staged in
-// shared memory per step, 4 x 4 outputs per thread accumulated in fp32 in row order
-// (deterministic).  CUDA cores: the tensor-core version is the next step.
-constexpr int kWgT = 64, kWgK = 16;
-__global__ void __launch_bounds__(256, 1) wgrad_kernel(const __nv_bfloat16* __restrict__ A,
-                                                    const __nv_bfloat16* __restrict__ B,
-                                                    const int32_t* __restrict__ offsets, int M,
-                                                    int N, float* __restrict__ out) {
-  __shared__ __align__(16) float sa[kWgK][kWgT];
-  __shared__ __align__(16) float sb[kWgK][kWgT];
-  const int e = blockIdx.z;
-  const int m0 = blockIdx.y * kWgT, n0 = blockIdx.x * kWgT;
-  const int r0 = __ldg(offsets + e), r1 = __ldg(offsets + e + 1);
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.0f;
-  for (int r = r0; r < r1; r += kWgK) {
-    for (int i = threadIdx.x; i < kWgK * kWgT; i += 256) {
-      const int rr = i / kWgT, cc = i % kWgT, row = r + rr;
-      const bool in = row < r1;
-      sa[rr][cc] = in ? __bfloat162float(A[static_cast<size_t>(row) * M + m0 + cc]) : 0.0f;
-      sb[rr][cc] = in ? __bfloat162float(B[static_cast<size_t>(row) * N + n0 + cc]) : 0.0f;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int rr = 0; rr < kWgK; ++rr) {
-      const float4 a = *reinterpret_cast<const float4*>(&sa[rr][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&sb[rr][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float* o = out + (static_cast<size_t>(e) * M + m0 + ty * 4 + i) * N + n0 + tx * 4;
-    *reinterpret_cast<float4*>(o) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
-  }
-}
-
 __global__ void fill_kernel(float* __restrict__ p, size_t n, float v) {
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -291,15 +245,6 @@ cudaError_t launch_swiglu_backward(const void* G, const void* dh, int S, int I, 
   swiglu_backward_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(G), static_cast<const __nv_bfloat16*>(dh), S, I,
       static_cast<__nv_bfloat16*>(dG));
-  return cudaGetLastError();
-}
-
-cudaError_t launch_wgrad(const void* A, const void* B, const int32_t* offsets, int E, int M,
-                         int N, float* out, cudaStream_t s) {
-  const dim3 grid(N / kWgT, M / kWgT, E);
-  count_launch();
-  wgrad_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(A),
-                                    static_cast<const __nv_bfloat16*>(B), offsets, M, N, out);
   return cudaGetLastError();
 }
 

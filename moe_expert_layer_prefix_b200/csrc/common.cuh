@@ -25,6 +25,7 @@ enum Site : int {
   SITE_GEMM_DRAIN = 106,     // loader draining its in-flight copies after an abort
   SITE_GEMM_AMAX = 107,      // linear-1 epilogue waiting for the other half's row amax
   SITE_GRID_BARRIER = 201,   // persistent kernel waiting at a grid-wide barrier
+  SITE_TILE_DEP = 202,       // persistent kernel waiting for the rows another CTA writes
   SITE_SCALE_FORMAT = 301,   // an fp32 block scale that is not a positive normal power of two
   SITE_SELFTEST_MBAR = 901,  // self-test: a wait on an mbarrier nothing ever arrives on
 };
@@ -293,6 +294,21 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f8f6f4 (no block scaling), E4M3 A and B, FP32 accumulator,
+// both K-major.
+__host__ __device__ constexpr uint32_t idesc_f8f6f4_e4m3(int M, int N) {
+  return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_f8f6f4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
 // Instruction descriptor, kind::mxf8f6f4 block-scaled, UE8M0 scales, both K-major.
 // Format codes: E4M3 = 0, E2M1 = 5.  The scale-factor byte selectors (bits [4,6) for B and
 // [29,31) for A) are OR-ed in per MMA.
@@ -465,6 +481,39 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expe
     __threadfence();
   }
   return __syncthreads_and(ok) != 0;
+}
+
+// Waits until the counter *c (written by other CTAs with a release, or after a fence) has
+// reached `target`, with acquire semantics.  Bounded like every wait: gives up after the
+// wait limit (or at once when *abort is raised), records MOE_ERR_TIMEOUT at SITE_TILE_DEP,
+// raises *abort and returns false.
+__device__ __forceinline__ bool wait_count(const uint32_t* c, uint32_t target, int* err,
+                                           volatile int* abort) {
+  if (ld_acquire_gpu(c) >= target) return true;
+  const long long t0 = clock64();
+  const long long limit = wait_limit(err);
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);  // leave the issue slots to the warps doing the work being waited for
+    if (ld_acquire_gpu(c) >= target) return true;
+    if ((it & 15u) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        report_error(err, MOE_ERR_TIMEOUT, SITE_TILE_DEP);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Publishes one unit of work to the counter *c after this warp's global stores: every lane
+// orders its stores (for generic readers, and for TMA readers through the proxy fence)
+// before lane 0's increment.
+__device__ __forceinline__ void publish_count(uint32_t* c, int lane) {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  __threadfence();
+  __syncwarp();
+  if (lane == 0) atomicAdd(c, 1u);
 }
 
 __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {

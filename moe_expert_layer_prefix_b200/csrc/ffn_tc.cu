@@ -1,6 +1,7 @@
 // Grouped expert GEMM kernel (gemm_tc.cuh holds the tensor-core pipeline and its source)
 // and its host-side launchers: tensor maps, tile-shape choice, cluster launch.
 #include "common.cuh"
+#include "gemm_promote.cuh"
 #include "gemm_tc.cuh"
 #include "internal.h"
 
@@ -68,7 +69,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   const Smem sm = carve<kCta, kTm>(smem_raw);
   gemm_init<kCta, kBlockScaled, kTm>(sm, &tmA, 1);
   if (threadIdx.x == 0) tma_prefetch_desc(&tmB);
-  gemm_prefix<kCta, kTm>(sm, p.offsets, p.E, p.n_tiles);
+  gemm_prefix<kCta, kTm>(sm, p.offsets, p.E);
   tc_fence_before();
   __syncthreads();
   if constexpr (kCta == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
@@ -81,6 +82,33 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if constexpr (kCta == 2) cluster_sync();
   tc_fence_after();
   gemm_fini<kCta>(sm);
+}
+
+// E4M3 x E4M3 with arbitrary fp32 block scales (gemm_promote.cuh).
+template <bool kSwiGLU, bool kOutE4M3>
+__global__ void __launch_bounds__(kThreads, 1)
+grouped_gemm_promote(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB, const TcParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const PSmem sm = pcarve(smem_raw);
+  pgemm_init(sm);
+  if (threadIdx.x == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  const Smem list{sm.sA, sm.sB, nullptr, sm.ss};
+  gemm_prefix<1, kBM>(list, p.offsets, p.E);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  pgemm_phase<kSwiGLU, kOutE4M3>(&tmA, &tmB, p, sm);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if ((threadIdx.x >> 5) == 1) {
+    __syncwarp();
+    tmem_dealloc(sm.ss->tmem_base, 256);
+  }
 }
 
 // ---------------------------------------------------------------------------------------
@@ -111,6 +139,9 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   p.out = a.out;
   p.out_scales = a.out_scales;
   p.err = a.err;
+  p.done = nullptr;
+  p.dep = nullptr;
+  p.dep_target = 0;
   auto kern = grouped_gemm_tc<kCta, kTm, kBS, kBFmt, kSw, kE4>;
   const size_t smem = Cfg<kCta, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -130,6 +161,41 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   cfg.numAttrs = 1;
   count_launch();
   return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p);
+}
+
+template <bool kSw, bool kE4>
+cudaError_t launch_promote(const FfnArgs& a, bool linear1, cudaStream_t s) {
+  const int K = linear1 ? a.H : a.I;
+  const int w_rows = linear1 ? 2 * a.I : a.H;
+  CUtensorMap tmA, tmB;
+  if (!make_kmajor_map(&tmA, a.a, static_cast<uint64_t>(a.S), static_cast<uint64_t>(K), 1, 128))
+    return cudaErrorInvalidValue;
+  // linear-1 loads the gate and the up half of a tile as two 64-row boxes
+  if (!make_kmajor_map(&tmB, a.w, static_cast<uint64_t>(a.E) * w_rows, static_cast<uint64_t>(K), 1,
+                       linear1 ? 64 : 128))
+    return cudaErrorInvalidValue;
+  TcParams p{};
+  p.offsets = a.offsets;
+  p.E = a.E;
+  p.S = a.S;
+  p.K = K;
+  p.n_tiles = linear1 ? a.I / 64 : a.H / 128;
+  p.w_rows = w_rows;
+  p.I = a.I;
+  p.n_out = linear1 ? a.I : a.H;
+  p.a_scales = a.a_scales;
+  p.b_scales = a.w_scales;
+  p.out = a.out;
+  p.out_scales = a.out_scales;
+  p.err = a.err;
+  auto kern = grouped_gemm_promote<kSw, kE4>;
+  const size_t smem = kPSmemBytes;
+  cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+  if (err != cudaSuccess) return err;
+  count_launch();
+  kern<<<num_sms(), kThreads, smem, s>>>(tmA, tmB, p);
+  return cudaGetLastError();
 }
 
 template <bool kBS, int kBFmt, bool kSw, bool kE4>
@@ -163,6 +229,10 @@ int gemm_tile_shape(int act, int S, int E, bool allow_pair) {
 
 cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s) {
   if (a.E > kMaxE) return cudaErrorNotSupported;
+  if (a.scale_fmt == MOE_SCALE_FP32) {
+    if (a.act != MOE_E4M3 || a.wt != MOE_E4M3) return cudaErrorNotSupported;
+    return launch_promote<true, true>(a, true, s);
+  }
   if (a.act == MOE_BF16 && a.wt == MOE_BF16) return launch_tc_any<false, 0, true, false>(a, true, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E4M3) return launch_tc_any<true, 0, true, true>(a, true, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E2M1) return launch_tc_any<true, 5, true, true>(a, true, s);
@@ -171,6 +241,10 @@ cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s) {
 
 cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s) {
   if (a.E > kMaxE) return cudaErrorNotSupported;
+  if (a.scale_fmt == MOE_SCALE_FP32) {
+    if (a.act != MOE_E4M3 || a.wt != MOE_E4M3) return cudaErrorNotSupported;
+    return launch_promote<false, false>(a, false, s);
+  }
   if (a.act == MOE_BF16 && a.wt == MOE_BF16) return launch_tc_any<false, 0, false, false>(a, false, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E4M3) return launch_tc_any<true, 0, false, false>(a, false, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E2M1) return launch_tc_any<true, 5, false, false>(a, false, s);

@@ -97,6 +97,13 @@ struct TcParams {
   void* out;
   float* out_scales;       // linear-1 with E4M3 h
   int* err;
+  // Tile-level dependencies inside one persistent launch (null in a standalone GEMM):
+  // every epilogue warp adds one to done[m-block] once its rows of a tile are stored, and
+  // the loaders of a tile wait until dep[m-block] reaches dep_target before reading its A
+  // rows (the rows the previous GEMM of the launch wrote).
+  uint32_t* done;
+  const uint32_t* dep;
+  uint32_t dep_target;
 };
 
 struct SharedState {
@@ -108,13 +115,15 @@ struct SharedState {
   uint64_t acc_full;
   uint64_t acc_empty;
   uint64_t drain;
+  uint64_t part_full[2];        // fp32-scale path: partial accumulator b written by the MMAs
+  uint64_t part_empty[2];       // ... and read out by every epilogue warp
   uint64_t amax_bar[4];         // linear-1 E4M3 epilogue: both column halves of a quadrant
                                 // have published their row's scale exponent
   int8_t ecode[2][2][kBM];      // [tile parity][column half][row of the tile]: the scale
                                 // exponent of the half's amax (kNoExp for an all-zero half)
   uint32_t tmem_base;
   int abort;
-  int total_tiles;
+  int mb_total;             // m-blocks over all experts (tiles = mb_total x n-blocks)
   int mb_start[kMaxE + 1];  // exclusive prefix of m-blocks per expert
   int offs[kMaxE + 1];
 };
@@ -294,10 +303,11 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
   }
 }
 
-// Tile list of one GEMM from the expert offsets (warp 3; the caller synchronises after).
+// m-block list of the expert offsets (warp 3; the caller synchronises after).  Every GEMM
+// over the same offsets and tile shape shares it (tile t = m-block t / n_tiles, n-block
+// t % n_tiles).
 template <int kCta, int kTm = kBM>
-__device__ __forceinline__ void gemm_prefix(const Smem& sm, const int32_t* offsets, int E,
-                                            int n_tiles) {
+__device__ __forceinline__ void gemm_prefix(const Smem& sm, const int32_t* offsets, int E) {
   using C = Cfg<kCta, kTm>;
   SharedState& ss = *sm.ss;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -321,7 +331,7 @@ __device__ __forceinline__ void gemm_prefix(const Smem& sm, const int32_t* offse
     carry += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
-  if (lane == 0) ss.total_tiles = ss.mb_start[E] * n_tiles;
+  if (lane == 0) ss.mb_total = ss.mb_start[E];
 }
 
 // Releases TMEM (warp 1); the caller synchronises the CTA (and the cluster) first.
@@ -357,7 +367,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
   constexpr int kElemsPerRow = kBlockScaled ? 128 : 64;  // K elements per stage
   const int KB = p.K / kElemsPerRow;
   const uint32_t tmem = ss.tmem_base;
-  const int total = ss.total_tiles;
+  const int total = ss.mb_total * p.n_tiles;
   volatile int* abort = &ss.abort;
 
   if (warp == 0) {
@@ -367,9 +377,15 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       constexpr uint32_t kCtaBytes = C::kATileBytes + kBBytes;
       uint32_t it = pipe.prod_it;
       const uint32_t it0 = it;
+      int dep_mb = -1;  // the last m-block whose A rows were found complete
       for (int t = cid; t < total && !*abort; t += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
         const int arow = tile.m0 + static_cast<int>(rank) * kTm;
+        if (p.dep != nullptr && t / p.n_tiles != dep_mb) {
+          dep_mb = t / p.n_tiles;
+          if (!wait_count(p.dep + dep_mb, p.dep_target, p.err, abort)) break;
+          fence_proxy_async_global();  // the rows other CTAs stored are read by TMA next
+        }
         // B rows of this CTA: linear-1 gate rows [nb*128, +128) then up rows [I + nb*128, +128);
         // linear-2 rows [nb*256, +256); a pair splits them between its two CTAs
         const int ebase = tile.e * p.w_rows;
@@ -552,13 +568,25 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       const uint32_t g0 = pipe.sf_it;
       uint32_t gi = g0;
       bool ok = true;
+      int dep_mb = -1;
       for (int lt = cid; lt < total && ok; lt += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
+        if (p.dep != nullptr && lt / p.n_tiles != dep_mb) {
+          // the A rows' scales are written by other CTAs' epilogues
+          dep_mb = lt / p.n_tiles;
+          if (!__all_sync(0xffffffffu, wait_count(p.dep + dep_mb, p.dep_target, p.err, abort))) {
+            ok = false;
+            break;
+          }
+        }
+        // only the tile's own rows are staged: the MMA's other rows (past the expert's end,
+        // or past a small tile's 32) are never stored, and their scales may not exist yet
+        uint32_t arow_ok = 0;
 #pragma unroll
         for (int r1 = 0; r1 < 4; ++r1) {
-          int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * r1;
-          m = m < p.S ? m : p.S - 1;  // rows past S are zero-filled by TMA; any scale will do
-          pa[r1] = p.a_scales + static_cast<size_t>(m) * KS;
+          const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * r1;
+          if (lane + 32 * r1 < kTm && m < tile.m_end) arow_ok |= 1u << r1;
+          pa[r1] = p.a_scales + static_cast<size_t>(m < p.S ? m : p.S - 1) * KS;
         }
         const int wr0 = kSwiGLU ? tile.nb * 128 : tile.nb * kBN;     // first B row, atom 0
         const int wr1 = kSwiGLU ? p.I + tile.nb * 128 : wr0 + 128;   // first B row, atom 1
@@ -595,6 +623,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           const bool whole = nk == 4;
 #pragma unroll
           for (int r1 = 0; r1 < 4; ++r1) {
+            if (!(arow_ok & (1u << r1))) continue;
             uint8_t* dst = sf + 16 * (lane + 32 * r1);
             const float* src = pa[r1] + 4 * g;
             if (a16 && whole) {
@@ -647,9 +676,19 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       const uint32_t g0 = pipe.sf_it;
       const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
       uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
+      uint32_t arow_ok = 0;  // rows of the current tile this lane converts (as the loader)
       for (int i = 0; i < n_grp; ++i) {
         const uint32_t gi = g0 + static_cast<uint32_t>(i);
         const int slot = static_cast<int>(gi % kSfGroups);
+        if (i % NG == 0) {
+          const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, cid + (i / NG) * ncl);
+          arow_ok = 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * c;
+            if (lane + 32 * c < kTm && m < tile.m_end) arow_ok |= 1u << c;
+          }
+        }
         if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfGroups) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort))
           break;
         uint8_t* sf = sSF + slot * kSfSlotBytes;
@@ -665,7 +704,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           for (int j = 0; j < 4; ++j) {
             if (j < nk) {
               w |= ((x[j] >> 23) & 0xFFu) << (8 * j);
-              bad |= not_pow2_scale(x[j]);
+              if (arow_ok & (1u << c)) bad |= not_pow2_scale(x[j]);
             }
           }
           wa[c] = w;
@@ -839,6 +878,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
                                           128 * half),
             static_cast<size_t>(p.n_out) * 2, rows_ok, chunks_ok, lane);
       }
+      if (p.done != nullptr) publish_count(p.done + t / p.n_tiles, lane);
       ++tiles;
     }
     pipe.hq = hq;

@@ -45,8 +45,15 @@ cudaError_t launch_gate_backward(const float* logits, const int32_t* topk_idx,
                                  int renorm, float scale, float* dlogits, cudaStream_t s);
 cudaError_t launch_swiglu_backward(const void* G, const void* dh, int S, int I, void* dG,
                                    cudaStream_t s);
-cudaError_t launch_wgrad(const void* A, const void* B, const int32_t* offsets, int E, int M,
-                         int N, float* out, cudaStream_t s);
+// Weight gradients on tensor cores (wgrad_tc.cu): pk = expert-padded segment starts, the
+// slot-major operands transposed into [C, wgrad_pad_cols(S, E)] copies, then the GEMM.
+size_t wgrad_pad_cols(int S, int E);
+cudaError_t launch_wgrad_pad_offsets(const int32_t* offsets, int E, int32_t* pk, cudaStream_t s);
+cudaError_t launch_pad_transpose(const void* X, int S, int C, const int32_t* offsets,
+                                 const int32_t* pk, int E, void* Xt, cudaStream_t s);
+cudaError_t launch_wgrad_tc(const void* At, const void* Bt, const int32_t* offsets,
+                            const int32_t* pk, int S, int E, int M, int N, float* out, int* err,
+                            cudaStream_t s);
 cudaError_t launch_fill(float* p, size_t n, float v, cudaStream_t s);
 
 struct FfnArgs {
@@ -60,6 +67,7 @@ struct FfnArgs {
   void* out;                   // h (linear-1) or y (linear-2)
   float* out_scales;           // h_scales (linear-1, E4M3) or null
   int* err;                    // device error word
+  int scale_fmt = MOE_SCALE_POW2;  // moe_scale_fmt of the fp32 block scales
 };
 
 cudaError_t launch_linear1_simt(const FfnArgs& a, cudaStream_t s);
@@ -103,8 +111,12 @@ struct ForwardArgs {
   void* y;
   void* out;
   uint32_t* bar;     // grid barrier words (zeroed by the launcher)
+  uint32_t* counters;  // 2 x forward_mb_cap(S, E) per-m-block completion counters
   int* err;
 };
+// m-blocks a persistent launch can have at most: the 32-row tiles' count for S slots over
+// E experts (each expert adds at most one partial block).
+inline int forward_mb_cap(int S, int E) { return (S + 31) / 32 + E; }
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s);
 
 // Self-test kernels whose bounded waits run out by construction (selftest.cu).

@@ -81,6 +81,17 @@ def test_argument_errors_need_no_gpu():
     assert M.moe_status_string(st) == "MOE_ERR_UNSUPPORTED"
 
 
+def test_scale_format_checked_before_launch():
+    import ctypes
+    fake = ctypes.c_void_p(1 << 20)
+    for fmt, act, wt, want in ((7, 2, 2, "MOE_ERR_INVALID_ARG"), (1, 2, 3, "MOE_ERR_UNSUPPORTED"),
+                               (1, 1, 1, "MOE_ERR_UNSUPPORTED")):
+        W = M.MoeWeights(act, wt, fake, fake, fake, fake, fmt)
+        st = M._linear1(fake, fake, fake, 256, 256, 128, 4, ctypes.byref(W), fake, fake, None, 0,
+                        None)
+        assert M.moe_status_string(st) == want, (fmt, act, wt)
+
+
 def test_wait_limit_and_selftest_arguments_checked_before_any_device_call():
     assert M.moe_status_string(M._set_wait_limit(-1)) == "MOE_ERR_INVALID_ARG"
     assert M.moe_status_string(M._selftest_wait(7, None)) == "MOE_ERR_INVALID_ARG"
