@@ -198,7 +198,6 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       b += h_bytes(S, I, act);
       b += round256(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));  // y
       b += 256;                                                               // grid barrier
-      b += round256(static_cast<size_t>(forward_mb_cap(S, E)) * 2 * 4);       // tile counters
       return b;
     }
     default:
@@ -414,8 +413,6 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
   void* ffn_ws = take(h_bytes(S, I, act));
   void* y = take(static_cast<size_t>(S) * H * (act == MOE_F32 ? 4 : 2));
   uint32_t* bar = reinterpret_cast<uint32_t*>(take(256));
-  uint32_t* counters =
-      reinterpret_cast<uint32_t*>(take(static_cast<size_t>(forward_mb_cap(S, E)) * 2 * 4));
   if (topk_idx_out) topk_idx = topk_idx_out;
   if (topk_w_out) topk_w = topk_w_out;
   if (offsets_out) offsets = offsets_out;
@@ -463,7 +460,6 @@ moe_status moe_forward_ex(const void* x, const float* x_scales, const float* log
     fa.y = y;
     fa.out = out;
     fa.bar = bar;
-    fa.counters = counters;
     fa.err = device_error_word();
     return cuda_status(launch_forward_fused(fa, stream));
   }

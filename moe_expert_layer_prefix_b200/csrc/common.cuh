@@ -25,7 +25,6 @@ enum Site : int {
   SITE_GEMM_DRAIN = 106,     // loader draining its in-flight copies after an abort
   SITE_GEMM_AMAX = 107,      // linear-1 epilogue waiting for the other half's row amax
   SITE_GRID_BARRIER = 201,   // persistent kernel waiting at a grid-wide barrier
-  SITE_TILE_DEP = 202,       // persistent kernel waiting for the rows another CTA writes
   SITE_SCALE_FORMAT = 301,   // an fp32 block scale that is not a positive normal power of two
   SITE_SELFTEST_MBAR = 901,  // self-test: a wait on an mbarrier nothing ever arrives on
 };
@@ -129,6 +128,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
       if (*abort) return false;
       if (clock64() - t0 > limit) {
         report_error(err, MOE_ERR_TIMEOUT, site);
+        *abort = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// A counter in shared memory published by one warp (release) and polled by another
+// (acquire): the hand-off from the GEMM's stager warp to its MMA-issuing thread.
+__device__ __forceinline__ void st_release_shared(uint32_t* p, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+// Polls the counter until it reaches `target`; bounded like mbar_wait (gives up after the
+// wait limit or once *abort is raised, recording MOE_ERR_TIMEOUT at SITE_GEMM_FULL).
+__device__ __forceinline__ bool wait_ready(const uint32_t* p, uint32_t target, int* err,
+                                           volatile int* abort) {
+  if (ld_acquire_shared(p) >= target) return true;
+  const long long t0 = clock64();
+  const long long limit = wait_limit(err);
+  for (uint32_t it = 1;; ++it) {
+    if (ld_acquire_shared(p) >= target) return true;
+    if ((it & 255u) == 0) {
+      if (*abort) return false;
+      if (clock64() - t0 > limit) {
+        report_error(err, MOE_ERR_TIMEOUT, SITE_GEMM_FULL);
         *abort = 1;
         return false;
       }
@@ -481,39 +512,6 @@ __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expe
     __threadfence();
   }
   return __syncthreads_and(ok) != 0;
-}
-
-// Waits until the counter *c (written by other CTAs with a release, or after a fence) has
-// reached `target`, with acquire semantics.  Bounded like every wait: gives up after the
-// wait limit (or at once when *abort is raised), records MOE_ERR_TIMEOUT at SITE_TILE_DEP,
-// raises *abort and returns false.
-__device__ __forceinline__ bool wait_count(const uint32_t* c, uint32_t target, int* err,
-                                           volatile int* abort) {
-  if (ld_acquire_gpu(c) >= target) return true;
-  const long long t0 = clock64();
-  const long long limit = wait_limit(err);
-  for (uint32_t it = 1;; ++it) {
-    __nanosleep(64);  // leave the issue slots to the warps doing the work being waited for
-    if (ld_acquire_gpu(c) >= target) return true;
-    if ((it & 15u) == 0) {
-      if (*abort) return false;
-      if (clock64() - t0 > limit) {
-        report_error(err, MOE_ERR_TIMEOUT, SITE_TILE_DEP);
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// Publishes one unit of work to the counter *c after this warp's global stores: every lane
-// orders its stores (for generic readers, and for TMA readers through the proxy fence)
-// before lane 0's increment.
-__device__ __forceinline__ void publish_count(uint32_t* c, int lane) {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-  __threadfence();
-  __syncwarp();
-  if (lane == 0) atomicAdd(c, 1u);
 }
 
 __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err) {

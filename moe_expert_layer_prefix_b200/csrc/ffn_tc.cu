@@ -139,9 +139,6 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   p.out = a.out;
   p.out_scales = a.out_scales;
   p.err = a.err;
-  p.done = nullptr;
-  p.dep = nullptr;
-  p.dep_target = 0;
   auto kern = grouped_gemm_tc<kCta, kTm, kBS, kBFmt, kSw, kE4>;
   const size_t smem = Cfg<kCta, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -52,9 +52,6 @@ struct FwdParams {
   void* out;
   uint32_t* bar;
   int* err;
-  uint32_t* cnt1;   // per m-block: linear-1 epilogue warps done (h rows stored)
-  uint32_t* cnt2;   // per m-block: linear-2 epilogue warps done (y rows stored)
-  int mb_cap;       // length of each counter array
   TcParams l1, l2;
 };
 
@@ -86,14 +83,9 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   int32_t* soffs = reinterpret_cast<int32_t*>(scratch + nwarps * kMaxE * 4 + 32 * 33 * 4);
   int32_t* wsum = soffs + 1028;
 
-  // A grid barrier or a tile dependency that timed out (recorded in the error word) ends
-  // the phases for this CTA: it releases TMEM and returns; the other CTAs give up at their
-  // next wait.
+  // A grid barrier that timed out (recorded in the error word) ends the phases for this
+  // CTA: it releases TMEM and returns; the other CTAs give up at their next barrier.
   do {
-    // 0. clear the per-m-block completion counters (made visible by the barriers below)
-    for (int i = blockIdx.x * kThreads + threadIdx.x; i < 2 * p.mb_cap; i += gridDim.x * kThreads)
-      (i < p.mb_cap ? p.cnt1 : p.cnt2)[i % p.mb_cap] = 0u;
-
     // 1. route: one warp per token
     if (p.E <= 256) {
       for (int t = gw; t < p.T; t += GW)
@@ -139,49 +131,33 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     fence_proxy_async_global();  // x_perm is read by TMA next
     if (!grid_sync(p.bar, p.err)) break;
 
-    // 7. linear-1 + SwiGLU + requantisation, then 8. linear-2, with no barrier between them:
-    //    the m-block list is computed once, every role moves on to linear-2 as soon as it is
-    //    done with linear-1, and a linear-2 tile's loaders wait only for the m-block of h
-    //    rows it reads (all n-blocks of that m-block stored by linear-1's epilogues, counted
-    //    in cnt1); linear-2's epilogues count their stored y rows in cnt2 for the combine.
+    // 7. linear-1 + SwiGLU + requantisation.  The m-block list is computed once for both
+    //    GEMMs (the same offsets and tile shape).
     Pipe pipe;
     gemm_prefix<1, kTm>(sm, p.offsets, p.E);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     gemm_phase<1, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
-    gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
-    if (sm.ss->abort) break;
+    fence_proxy_async_global();  // h is read by TMA next
+    if (!grid_sync(p.bar, p.err)) break;
 
-    // 9. combine, token by token once the y rows of its k slots are stored (each slot's
-    //    m-block counted complete in cnt2).  A warp keeps two 16-byte loads per lane and
-    //    source row in flight and takes a whole token when there are tokens enough for
-    //    every warp; fewer tokens are split into 512-column chunks.
-    const SharedState& ss = *sm.ss;
-    const uint32_t y_target = static_cast<uint32_t>(p.l2.n_tiles) * kEpiWarps;
-    volatile int* abort = &sm.ss->abort;
-    auto token_ready = [&](int t) {
-      bool ok = true;
-      if (lane < p.k) {
-        const int e = __ldcg(p.topk_idx + static_cast<size_t>(t) * p.k + lane);
-        const int slot = __ldcg(p.slot_of + static_cast<size_t>(t) * p.k + lane);
-        const int mb = ss.mb_start[e] + (slot - ss.offs[e]) / Cfg<1, kTm>::kTileM;
-        ok = wait_count(p.cnt2 + mb, y_target, p.err, abort);
-      }
-      return __all_sync(0xffffffffu, ok);
-    };
+    // 8. linear-2
+    gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
+    if (!grid_sync(p.bar, p.err)) break;
+
+    // 9. combine.  A warp keeps two 16-byte loads per lane and source row in flight and
+    //    takes a whole token when there are tokens enough for every warp; fewer tokens are
+    //    split into 512-column chunks.
     if (p.T >= 2 * GW) {
-      for (int t = gw; t < p.T; t += GW) {
-        if (!token_ready(t)) break;
+      for (int t = gw; t < p.T; t += GW)
         combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, 0, p.H / 8);
-      }
     } else {
       const int nc = combine_chunks<2>(p.H);
       const int width = nc == 1 ? p.H / 8 : 64;
       const long items = static_cast<long>(p.T) * nc;
       for (long it = gw; it < items; it += GW) {
         const int t = static_cast<int>(it / nc), c = static_cast<int>(it % nc);
-        if (!token_ready(t)) break;
         combine_token<false, 2>(p.y, p.slot_of, p.topk_w, t, p.k, p.H, p.out, lane, c * width,
                                 (c + 1) * width);
       }
@@ -235,9 +211,6 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   p.out = a.out;
   p.bar = a.bar;
   p.err = a.err;
-  p.mb_cap = forward_mb_cap(S, a.E);
-  p.cnt1 = a.counters;
-  p.cnt2 = a.counters + p.mb_cap;
   TcParams l1{}, l2{};
   l1.offsets = l2.offsets = a.offsets;
   l1.E = l2.E = a.E;
@@ -260,11 +233,6 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   l2.b_scales = a.w2_scales;
   l2.out = a.y;
   l2.out_scales = nullptr;
-  l1.done = p.cnt1;
-  l1.dep = nullptr;
-  l2.done = p.cnt2;
-  l2.dep = p.cnt1;
-  l2.dep_target = static_cast<uint32_t>(l1.n_tiles) * kEpiWarps;
   p.l1 = l1;
   p.l2 = l2;
 

@@ -22,11 +22,14 @@
 //               CTAs' copies complete on the leader's stage barrier
 //   warp 1      MMA issuer (one thread, leader CTA): tcgen05.mma 128|256 x 256 x {16|32}
 //               into a TMEM fp32 accumulator (256 columns); tcgen05.commit frees ring stages
-//               (in both CTAs of a pair)
-//   warp 2      scale loader (block-scaled kinds): copies the raw scale words of each k-step
-//               into a 16-slot shared-memory ring with asynchronous 4-byte copies (cp.async)
-//   warp 3      scale converter: UE8M0 bytes in the layout tcgen05.cp reads, then signals the
-//               (leader's) slot barriers; before each GEMM phase it also builds the tile list
+//               (in both CTAs of a pair).  It waits on no stage barrier itself: it polls a
+//               shared-memory count of ready k-steps (an mbarrier wait costs the issuing
+//               thread about as much as the four MMAs of a k-step)
+//   warp 2      scale loader (block-scaled kinds): copies the raw scales of each group of 4
+//               k-steps into a 4-slot shared-memory ring with asynchronous copies (cp.async)
+//   warp 3      stager: UE8M0 bytes in the layout tcgen05.cp reads (block-scaled kinds), then
+//               waits for each k-step's A/B stage and publishes the ready count; before each
+//               GEMM phase it also builds the tile list
 //   warps 4..11 epilogue: two warps per TMEM lane quadrant (warp w reads lanes
 //               32(w%4)..+31, one output row per thread), each taking half of the tile's
 //               columns, so that the accumulator is read out in a quarter of the time and
@@ -97,13 +100,6 @@ struct TcParams {
   void* out;
   float* out_scales;       // linear-1 with E4M3 h
   int* err;
-  // Tile-level dependencies inside one persistent launch (null in a standalone GEMM):
-  // every epilogue warp adds one to done[m-block] once its rows of a tile are stored, and
-  // the loaders of a tile wait until dep[m-block] reaches dep_target before reading its A
-  // rows (the rows the previous GEMM of the launch wrote).
-  uint32_t* done;
-  const uint32_t* dep;
-  uint32_t dep_target;
 };
 
 struct SharedState {
@@ -124,6 +120,8 @@ struct SharedState {
   uint32_t tmem_base;
   int abort;
   int mb_total;             // m-blocks over all experts (tiles = mb_total x n-blocks)
+  uint32_t ready;           // stager -> MMA issuer: k-steps whose A/B stage (and scales) are
+                            // in shared memory, counted over the whole launch
   int mb_start[kMaxE + 1];  // exclusive prefix of m-blocks per expert
   int offs[kMaxE + 1];
 };
@@ -246,6 +244,7 @@ struct Pipe {
   uint32_t sf_it = 0;    // scale loader / converter: groups of 4 k-steps staged
   uint32_t sf_grp = 0;   // MMA issuer: groups of 4 k-steps whose scales were copied to TMEM
   uint32_t hq = 0;       // epilogue: linear-1 tiles requantised to E4M3 (amax exchanges)
+  uint32_t st_it = 0;    // stager: k-steps published as ready
 };
 
 // Shared-memory carve-up (1024-byte aligned; identical offsets in both CTAs of a pair).
@@ -289,6 +288,7 @@ __device__ __forceinline__ void gemm_init(const Smem& sm, const CUtensorMap* tma
     mbar_init(&ss.drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&ss.amax_bar[q], 64);  // every lane of both halves
     ss.abort = 0;
+    ss.ready = 0;
     fence_barrier_init();
     for (int i = 0; i < ntmaps; ++i) tma_prefetch_desc(tmaps + i);
   }
@@ -377,15 +377,9 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       constexpr uint32_t kCtaBytes = C::kATileBytes + kBBytes;
       uint32_t it = pipe.prod_it;
       const uint32_t it0 = it;
-      int dep_mb = -1;  // the last m-block whose A rows were found complete
       for (int t = cid; t < total && !*abort; t += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
         const int arow = tile.m0 + static_cast<int>(rank) * kTm;
-        if (p.dep != nullptr && t / p.n_tiles != dep_mb) {
-          dep_mb = t / p.n_tiles;
-          if (!wait_count(p.dep + dep_mb, p.dep_target, p.err, abort)) break;
-          fence_proxy_async_global();  // the rows other CTAs stored are read by TMA next
-        }
         // B rows of this CTA: linear-1 gate rows [nb*128, +128) then up rows [I + nb*128, +128);
         // linear-2 rows [nb*256, +256); a pair splits them between its two CTAs
         const int ebase = tile.e * p.w_rows;
@@ -447,8 +441,10 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           const int stage = static_cast<int>(it % kStages);
-          const uint32_t phase = (it / kStages) & 1u;
-          if (!mbar_wait<kPair>(&ss.full[stage], phase, p.err, SITE_GEMM_FULL, abort)) {
+          // the stager warp has seen this k-step's stage land (and converted its scales):
+          // a shared-memory poll here instead of an mbarrier wait, which costs the issuing
+          // thread far more than the MMAs' own issue
+          if (!wait_ready(&ss.ready, it + 1u, p.err, abort)) {
             ok = false;
             break;
           }
@@ -458,15 +454,6 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           // once its first k-step has passed)
           const uint32_t gcur = grp_start ? grp : grp - 1u;
           const int slot = static_cast<int>(gcur % kSfGroups);
-          if constexpr (kBlockScaled) {
-            if (grp_start) {
-              if (!mbar_wait<kPair>(&ss.sf_full[slot], (gcur / kSfGroups) & 1u, p.err,
-                                    SITE_GEMM_FULL, abort)) {
-                ok = false;
-                break;
-              }
-            }
-          }
           tc_fence_after();
           const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * C::kATileBytes));
           const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
@@ -568,17 +555,8 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       const uint32_t g0 = pipe.sf_it;
       uint32_t gi = g0;
       bool ok = true;
-      int dep_mb = -1;
       for (int lt = cid; lt < total && ok; lt += ncl) {
         const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
-        if (p.dep != nullptr && lt / p.n_tiles != dep_mb) {
-          // the A rows' scales are written by other CTAs' epilogues
-          dep_mb = lt / p.n_tiles;
-          if (!__all_sync(0xffffffffu, wait_count(p.dep + dep_mb, p.dep_target, p.err, abort))) {
-            ok = false;
-            break;
-          }
-        }
         // only the tile's own rows are staged: the MMA's other rows (past the expert's end,
         // or past a small tile's 32) are never stored, and their scales may not exist yet
         uint32_t arow_ok = 0;
@@ -659,104 +637,131 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       pipe.sf_it = g0 + static_cast<uint32_t>(my_tiles * NG);
     }
   } else if (warp == 3) {
-    // ------------------------------------------------------------------ scale converter
-    // Rewrites each staged group in place into the layout tcgen05.cp reads: per 128-row
-    // atom, 32 lines of 16 bytes, line l word c for row 32c + l, one UE8M0 per byte.  A and
-    // E4M3 B scales cover 128 of K, so byte j of a word is k-step j of the group (one TMEM
-    // copy per group; the MMA's scale-byte selector picks the k-step); the UE8M0 byte of a
-    // power-of-two fp32 scale is its exponent field.  E2M1 B scales are per 32 of K and
-    // already UE8M0: each k-step gets its own 2 atoms (byte = sub-block).  Lane l reads only
-    // rows congruent to l mod 32 and writes only lines that held such rows, so the in-place
-    // rewrite needs no exchange between lanes.  A scale word that is not a positive normal
-    // power of two (no exact UE8M0 byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
-    if constexpr (kBlockScaled) {
-      const int NG = (KB + 3) / 4;
-      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
-      const int n_grp = my_tiles * NG;
-      const uint32_t g0 = pipe.sf_it;
-      const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
-      uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
-      uint32_t arow_ok = 0;  // rows of the current tile this lane converts (as the loader)
-      for (int i = 0; i < n_grp; ++i) {
-        const uint32_t gi = g0 + static_cast<uint32_t>(i);
-        const int slot = static_cast<int>(gi % kSfGroups);
-        if (i % NG == 0) {
-          const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, cid + (i / NG) * ncl);
-          arow_ok = 0;
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * c;
-            if (lane + 32 * c < kTm && m < tile.m_end) arow_ok |= 1u << c;
-          }
-        }
-        if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfGroups) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort))
-          break;
-        uint8_t* sf = sSF + slot * kSfSlotBytes;
-        const int nk = min(4, KB - 4 * (i % NG));
-        // A: rows lane + 32c -> line lane
-        uint32_t wa[4];
+    // ------------------------------------------------------------------ stager
+    // Walks this CTA's k-steps in the MMA issuer's order.  At a group's first k-step of a
+    // block-scaled kind it rewrites the group's staged raw scales in place into the layout
+    // tcgen05.cp reads: per 128-row atom, 32 lines of 16 bytes, line l word c for row
+    // 32c + l, one UE8M0 per byte.  A and E4M3 B scales cover 128 of K, so byte j of a word
+    // is k-step j of the group (one TMEM copy per group; the MMA's scale-byte selector picks
+    // the k-step); the UE8M0 byte of a power-of-two fp32 scale is its exponent field.  E2M1 B
+    // scales are per 32 of K and already UE8M0: each k-step gets its own 2 atoms (byte =
+    // sub-block).  Lane l reads only rows congruent to l mod 32 and writes only lines that
+    // held such rows, so the in-place rewrite needs no exchange between lanes.  Then it waits
+    // for the k-step's A/B stage to land and publishes the count of ready k-steps, which the
+    // MMA issuer polls: the mbarrier waits run here, off the issuing thread.  In a pair both
+    // CTAs convert their own scales and the leader's stager waits for the peer's before
+    // publishing.  A scale word that is not a positive normal power of two (no exact UE8M0
+    // byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
+    const int NG = (KB + 3) / 4;
+    uint32_t it = pipe.st_it;  // k-steps, the MMA issuer's sequence
+    uint32_t gi = pipe.sf_it;  // groups, the scale loader's sequence
+    const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
+    uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
+    bool ok = true;
+    for (int lt = cid; lt < total && ok; lt += ncl) {
+      uint32_t arow_ok = 0;  // rows of this tile this lane converts (as the loader staged them)
+      if constexpr (kBlockScaled) {
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(sf + 16 * (lane + 32 * c));
-          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-          uint32_t w = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < nk) {
-              w |= ((x[j] >> 23) & 0xFFu) << (8 * j);
-              if (arow_ok & (1u << c)) bad |= not_pow2_scale(x[j]);
-            }
-          }
-          wa[c] = w;
-        }
-        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
-        if constexpr (kBFmt == 5) {
-          // rows 128a + 32c + lane, 16 B each (k-step j = word j) -> line (k-step j, atom a)
-          uint4 v[2][4];
-#pragma unroll
-          for (int a = 0; a < 2; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              v[a][c] = *reinterpret_cast<const uint4*>(sf + kSfBOff + 16 * (128 * a + 32 * c + lane));
-#pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int a = 0; a < 2; ++a) {
-              const uint32_t w0 = j == 0 ? v[a][0].x : j == 1 ? v[a][0].y : j == 2 ? v[a][0].z : v[a][0].w;
-              const uint32_t w1 = j == 0 ? v[a][1].x : j == 1 ? v[a][1].y : j == 2 ? v[a][1].z : v[a][1].w;
-              const uint32_t w2 = j == 0 ? v[a][2].x : j == 1 ? v[a][2].y : j == 2 ? v[a][2].z : v[a][2].w;
-              const uint32_t w3 = j == 0 ? v[a][3].x : j == 1 ? v[a][3].y : j == 2 ? v[a][3].z : v[a][3].w;
-              *reinterpret_cast<uint4*>(sf + kSfBOff + 1024 * j + 512 * a + 16 * lane) =
-                  make_uint4(w0, w1, w2, w3);
-            }
-        } else {
-          // the two weight blocks' scales, the same for every row of their atom
-          const uint4 rg = *reinterpret_cast<const uint4*>(sf + kSfBRawE4);
-          const uint4 ru = *reinterpret_cast<const uint4*>(sf + kSfBRawE4 + 16);
-          const uint32_t xg[4] = {rg.x, rg.y, rg.z, rg.w}, xu[4] = {ru.x, ru.y, ru.z, ru.w};
-          uint32_t wb0 = 0, wb1 = 0;
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            if (j < nk) {
-              wb0 |= ((xg[j] >> 23) & 0xFFu) << (8 * j);
-              wb1 |= ((xu[j] >> 23) & 0xFFu) << (8 * j);
-              bad |= not_pow2_scale(xg[j]) | not_pow2_scale(xu[j]);
-            }
-          }
-          *reinterpret_cast<uint4*>(sf + kSfBOff + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
-          *reinterpret_cast<uint4*>(sf + kSfBOff + 512 + 16 * lane) = make_uint4(wb1, wb1, wb1, wb1);
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) {
-          if constexpr (kPair) mbar_arrive_cluster(full_lead0 + slot * sizeof(uint64_t));
-          else mbar_arrive(&ss.sf_full[slot]);
+          const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * c;
+          if (lane + 32 * c < kTm && m < tile.m_end) arow_ok |= 1u << c;
         }
       }
-      pipe.sf_it = g0 + static_cast<uint32_t>(n_grp);
-      // the exponent fields were used all the same: the result is undefined, the call fails
-      if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        if constexpr (kBlockScaled) {
+          if ((kb & 3) == 0) {
+            const int slot = static_cast<int>(gi % kSfGroups);
+            if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfGroups) & 1u, p.err, SITE_GEMM_SF_EMPTY,
+                           abort)) {
+              ok = false;
+              break;
+            }
+            uint8_t* sf = sSF + slot * kSfSlotBytes;
+            const int nk = min(4, KB - kb);
+            // A: rows lane + 32c -> line lane
+            uint32_t wa[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              const uint4 v = *reinterpret_cast<const uint4*>(sf + 16 * (lane + 32 * c));
+              const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+              uint32_t w = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (j < nk) {
+                  w |= ((x[j] >> 23) & 0xFFu) << (8 * j);
+                  if (arow_ok & (1u << c)) bad |= not_pow2_scale(x[j]);
+                }
+              }
+              wa[c] = w;
+            }
+            *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+            if constexpr (kBFmt == 5) {
+              // rows 128a + 32c + lane, 16 B each (k-step j = word j) -> line (k-step j, atom a)
+              uint4 v[2][4];
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                  v[a][c] = *reinterpret_cast<const uint4*>(sf + kSfBOff + 16 * (128 * a + 32 * c + lane));
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                  const uint32_t w0 = j == 0 ? v[a][0].x : j == 1 ? v[a][0].y : j == 2 ? v[a][0].z : v[a][0].w;
+                  const uint32_t w1 = j == 0 ? v[a][1].x : j == 1 ? v[a][1].y : j == 2 ? v[a][1].z : v[a][1].w;
+                  const uint32_t w2 = j == 0 ? v[a][2].x : j == 1 ? v[a][2].y : j == 2 ? v[a][2].z : v[a][2].w;
+                  const uint32_t w3 = j == 0 ? v[a][3].x : j == 1 ? v[a][3].y : j == 2 ? v[a][3].z : v[a][3].w;
+                  *reinterpret_cast<uint4*>(sf + kSfBOff + 1024 * j + 512 * a + 16 * lane) =
+                      make_uint4(w0, w1, w2, w3);
+                }
+            } else {
+              // the two weight blocks' scales, the same for every row of their atom
+              const uint4 rg = *reinterpret_cast<const uint4*>(sf + kSfBRawE4);
+              const uint4 ru = *reinterpret_cast<const uint4*>(sf + kSfBRawE4 + 16);
+              const uint32_t xg[4] = {rg.x, rg.y, rg.z, rg.w}, xu[4] = {ru.x, ru.y, ru.z, ru.w};
+              uint32_t wb0 = 0, wb1 = 0;
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (j < nk) {
+                  wb0 |= ((xg[j] >> 23) & 0xFFu) << (8 * j);
+                  wb1 |= ((xu[j] >> 23) & 0xFFu) << (8 * j);
+                  bad |= not_pow2_scale(xg[j]) | not_pow2_scale(xu[j]);
+                }
+              }
+              *reinterpret_cast<uint4*>(sf + kSfBOff + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
+              *reinterpret_cast<uint4*>(sf + kSfBOff + 512 + 16 * lane) =
+                  make_uint4(wb1, wb1, wb1, wb1);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if constexpr (kPair) {
+              if (lane == 0) mbar_arrive_cluster(full_lead0 + slot * sizeof(uint64_t));
+              if (rank == 0 && !mbar_wait<true>(&ss.sf_full[slot], (gi / kSfGroups) & 1u, p.err,
+                                                SITE_GEMM_FULL, abort)) {
+                ok = false;
+                break;
+              }
+            }
+            ++gi;
+          }
+        }
+        if (rank == 0) {
+          const int stage = static_cast<int>(it % kStages);
+          if (!mbar_wait<kPair>(&ss.full[stage], (it / kStages) & 1u, p.err, SITE_GEMM_FULL,
+                                abort)) {
+            ok = false;
+            break;
+          }
+          __syncwarp();
+          if (lane == 0) st_release_shared(&ss.ready, it + 1u);
+        }
+      }
     }
+    pipe.st_it = it;
+    pipe.sf_it = gi;
+    // the exponent fields were used all the same: the result is undefined, the call fails
+    if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant (the warp's 32 rows)
@@ -878,7 +883,6 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
                                           128 * half),
             static_cast<size_t>(p.n_out) * 2, rows_ok, chunks_ok, lane);
       }
-      if (p.done != nullptr) publish_count(p.done + t / p.n_tiles, lane);
       ++tiles;
     }
     pipe.hq = hq;

@@ -111,12 +111,8 @@ struct ForwardArgs {
   void* y;
   void* out;
   uint32_t* bar;     // grid barrier words (zeroed by the launcher)
-  uint32_t* counters;  // 2 x forward_mb_cap(S, E) per-m-block completion counters
   int* err;
 };
-// m-blocks a persistent launch can have at most: the 32-row tiles' count for S slots over
-// E experts (each expert adds at most one partial block).
-inline int forward_mb_cap(int S, int E) { return (S + 31) / 32 + E; }
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s);
 
 // Self-test kernels whose bounded waits run out by construction (selftest.cu).
