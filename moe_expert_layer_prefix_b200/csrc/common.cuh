@@ -147,21 +147,25 @@ __device__ __forceinline__ uint32_t ld_acquire_shared(const uint32_t* p) {
   return v;
 }
 
-// Polls the counter until it reaches `target`; bounded like mbar_wait (gives up after the
-// wait limit or once *abort is raised, recording MOE_ERR_TIMEOUT at SITE_GEMM_FULL).
-__device__ __forceinline__ bool wait_ready(const uint32_t* p, uint32_t target, int* err,
-                                           volatile int* abort) {
-  if (ld_acquire_shared(p) >= target) return true;
+// Polls the counter until it reaches `target` and returns the value seen (0 when it gave
+// up); bounded like mbar_wait (gives up after the wait limit or once *abort is raised,
+// recording MOE_ERR_TIMEOUT at SITE_GEMM_FULL).  A caller that keeps the returned value
+// needs no poll at all for the k-steps it already covers.
+__device__ __forceinline__ uint32_t wait_ready(const uint32_t* p, uint32_t target, int* err,
+                                               volatile int* abort) {
+  uint32_t v = ld_acquire_shared(p);
+  if (v >= target) return v;
   const long long t0 = clock64();
   const long long limit = wait_limit(err);
   for (uint32_t it = 1;; ++it) {
-    if (ld_acquire_shared(p) >= target) return true;
+    v = ld_acquire_shared(p);
+    if (v >= target) return v;
     if ((it & 255u) == 0) {
-      if (*abort) return false;
+      if (*abort) return 0;
       if (clock64() - t0 > limit) {
         report_error(err, MOE_ERR_TIMEOUT, SITE_GEMM_FULL);
         *abort = 1;
-        return false;
+        return 0;
       }
     }
   }

@@ -22,12 +22,15 @@
 //               CTAs' copies complete on the leader's stage barrier
 //   warp 1      MMA issuer (one thread, leader CTA): tcgen05.mma 128|256 x 256 x {16|32}
 //               into a TMEM fp32 accumulator (256 columns); tcgen05.commit frees ring stages
-//               (in both CTAs of a pair).  It waits on no stage barrier itself: it polls a
-//               shared-memory count of ready k-steps (an mbarrier wait costs the issuing
-//               thread about as much as the four MMAs of a k-step)
+//               (in both CTAs of a pair).  It waits on the stage barriers itself, except for
+//               E2M1 weights over K loops of 8 or more k-steps: there it polls a shared-
+//               memory count of ready k-steps that the stager publishes (an mbarrier wait
+//               costs the issuing thread about as much as the four MMAs of a k-step, and
+//               E2M1 adds two scale copies per k-step on the same thread)
 //   warp 2      scale loader (block-scaled kinds): copies the raw scales of each group of 4
 //               k-steps into a 4-slot shared-memory ring with asynchronous copies (cp.async)
-//   warp 3      stager: UE8M0 bytes in the layout tcgen05.cp reads (block-scaled kinds), then
+//   warp 3      scale converter (block-scaled kinds): UE8M0 bytes in the layout tcgen05.cp
+//               reads, one barrier arrival per group; as the stager (see warp 1) it also
 //               waits for each k-step's A/B stage and publishes the ready count; before each
 //               GEMM phase it also builds the tile list
 //   warps 4..11 epilogue: two warps per TMEM lane quadrant (warp w reads lanes
@@ -348,9 +351,12 @@ __device__ __forceinline__ void gemm_fini(const Smem& sm) {
 // kCta: 1 (single) or 2 (pair).  kBlockScaled: false -> BF16 kind::f16; true ->
 // kind::mxf8f6f4 with A = E4M3 and B = E4M3 (kBFmt 0) or E2M1 (kBFmt 5).  kSwiGLU: linear-1
 // epilogue, else linear-2.  kOutE4M3: linear-1 stores h as E4M3 + 1x128 scales (else BF16).
-template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm = kBM>
-__device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
-                                           const TcParams& p, const Smem& sm, Pipe& pipe) {
+// kStager: the MMA issuer polls the stager warp's ready count instead of waiting on the
+// stage barriers itself (E2M1 weights only; gemm_phase picks it).
+template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm,
+          bool kStager>
+__device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
+                                             const TcParams& p, const Smem& sm, Pipe& pipe) {
   using C = Cfg<kCta, kTm>;
   constexpr bool kPair = kCta == 2;
   constexpr int kStages = C::kStages;
@@ -366,6 +372,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
   const int ncl = kPair ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
   constexpr int kElemsPerRow = kBlockScaled ? 128 : 64;  // K elements per stage
   const int KB = p.K / kElemsPerRow;
+  static_assert(!kStager || kBlockScaled, "the stager converts block scales");
   const uint32_t tmem = ss.tmem_base;
   const int total = ss.mb_total * p.n_tiles;
   volatile int* abort = &ss.abort;
@@ -432,6 +439,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       constexpr uint32_t kIdesc = kBlockScaled ? idesc_mxf8f6f4(kMmaM, kBN, 0u, kBFmt)
                                                : idesc_bf16(kMmaM, kBN);
       uint32_t it = pipe.mma_it, tiles = pipe.tiles, grp = pipe.sf_grp;
+      uint32_t seen = 0;  // the stager's ready count as last observed
       bool issued_any = false;
       for (int t = cid; t < total && !*abort; t += ncl) {
         const uint32_t acc_phase = tiles & 1u;
@@ -441,12 +449,23 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
         bool ok = true;
         for (int kb = 0; kb < KB; ++kb) {
           const int stage = static_cast<int>(it % kStages);
-          // the stager warp has seen this k-step's stage land (and converted its scales):
-          // a shared-memory poll here instead of an mbarrier wait, which costs the issuing
-          // thread far more than the MMAs' own issue
-          if (!wait_ready(&ss.ready, it + 1u, p.err, abort)) {
-            ok = false;
-            break;
+          // with the stager: it has seen this k-step's stage land (and converted its
+          // scales); a shared-memory poll here instead of an mbarrier wait, which costs the
+          // issuing thread far more than the MMAs' own issue
+          if constexpr (kStager) {
+            if (seen < it + 1u) {
+              seen = wait_ready(&ss.ready, it + 1u, p.err, abort);
+              if (seen == 0) {
+                ok = false;
+                break;
+              }
+            }
+          } else {
+            if (!mbar_wait<kPair>(&ss.full[stage], (it / kStages) & 1u, p.err, SITE_GEMM_FULL,
+                                  abort)) {
+              ok = false;
+              break;
+            }
           }
           const bool grp_start = (kb & 3) == 0;
           const bool grp_end = (kb & 3) == 3 || kb == KB - 1;
@@ -454,6 +473,15 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
           // once its first k-step has passed)
           const uint32_t gcur = grp_start ? grp : grp - 1u;
           const int slot = static_cast<int>(gcur % kSfGroups);
+          if constexpr (kBlockScaled && !kStager) {
+            if (grp_start) {
+              if (!mbar_wait<kPair>(&ss.sf_full[slot], (gcur / kSfGroups) & 1u, p.err,
+                                    SITE_GEMM_FULL, abort)) {
+                ok = false;
+                break;
+              }
+            }
+          }
           tc_fence_after();
           const uint64_t adesc = desc_kmajor_sw128(smem_u32(sA + stage * C::kATileBytes));
           const uint64_t bdesc = desc_kmajor_sw128(smem_u32(sB + stage * C::kBTileBytes));
@@ -636,7 +664,7 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
       cp_async_wait_all();  // no copy may still be landing when the CTA moves on
       pipe.sf_it = g0 + static_cast<uint32_t>(my_tiles * NG);
     }
-  } else if (warp == 3) {
+  } else if (kStager && warp == 3) {
     // ------------------------------------------------------------------ stager
     // Walks this CTA's k-steps in the MMA issuer's order.  At a group's first k-step of a
     // block-scaled kind it rewrites the group's staged raw scales in place into the layout
@@ -652,7 +680,6 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     // CTAs convert their own scales and the leader's stager waits for the peer's before
     // publishing.  A scale word that is not a positive normal power of two (no exact UE8M0
     // byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
-    const int NG = (KB + 3) / 4;
     uint32_t it = pipe.st_it;  // k-steps, the MMA issuer's sequence
     uint32_t gi = pipe.sf_it;  // groups, the scale loader's sequence
     const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
@@ -742,6 +769,10 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
                 ok = false;
                 break;
               }
+            } else if (lane == 0) {
+              // nobody waits on it here, but a later phase without the stager (a short K
+              // loop in the persistent kernel) reads this slot's phase
+              mbar_arrive(&ss.sf_full[slot]);
             }
             ++gi;
           }
@@ -762,6 +793,108 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     pipe.sf_it = gi;
     // the exponent fields were used all the same: the result is undefined, the call fails
     if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
+  } else if (warp == 3) {
+    // ------------------------------------------------------------------ scale converter
+    // Rewrites each staged group in place into the layout tcgen05.cp reads: per 128-row
+    // atom, 32 lines of 16 bytes, line l word c for row 32c + l, one UE8M0 per byte.  A and
+    // E4M3 B scales cover 128 of K, so byte j of a word is k-step j of the group (one TMEM
+    // copy per group; the MMA's scale-byte selector picks the k-step); the UE8M0 byte of a
+    // power-of-two fp32 scale is its exponent field.  E2M1 B scales are per 32 of K and
+    // already UE8M0: each k-step gets its own 2 atoms (byte = sub-block).  Lane l reads only
+    // rows congruent to l mod 32 and writes only lines that held such rows, so the in-place
+    // rewrite needs no exchange between lanes.  A scale word that is not a positive normal
+    // power of two (no exact UE8M0 byte) is reported once at the end as MOE_ERR_UNSUPPORTED.
+    if constexpr (kBlockScaled) {
+      const int NG = (KB + 3) / 4;
+      const int my_tiles = total > cid ? (total - cid + ncl - 1) / ncl : 0;
+      const int n_grp = my_tiles * NG;
+      const uint32_t g0 = pipe.sf_it;
+      const uint32_t full_lead0 = mapa_shared(smem_u32(&ss.sf_full[0]), 0);
+      uint32_t bad = 0;  // a scale word that is not a positive normal power of two was seen
+      uint32_t arow_ok = 0;  // rows of the current tile this lane converts (as the loader)
+      for (int i = 0; i < n_grp; ++i) {
+        const uint32_t gi = g0 + static_cast<uint32_t>(i);
+        const int slot = static_cast<int>(gi % kSfGroups);
+        if (i % NG == 0) {
+          const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, cid + (i / NG) * ncl);
+          arow_ok = 0;
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * c;
+            if (lane + 32 * c < kTm && m < tile.m_end) arow_ok |= 1u << c;
+          }
+        }
+        if (!mbar_wait(&ss.sf_raw[slot], (gi / kSfGroups) & 1u, p.err, SITE_GEMM_SF_EMPTY, abort))
+          break;
+        uint8_t* sf = sSF + slot * kSfSlotBytes;
+        const int nk = min(4, KB - 4 * (i % NG));
+        // A: rows lane + 32c -> line lane
+        uint32_t wa[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(sf + 16 * (lane + 32 * c));
+          const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+          uint32_t w = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              w |= ((x[j] >> 23) & 0xFFu) << (8 * j);
+              if (arow_ok & (1u << c)) bad |= not_pow2_scale(x[j]);
+            }
+          }
+          wa[c] = w;
+        }
+        *reinterpret_cast<uint4*>(sf + 16 * lane) = make_uint4(wa[0], wa[1], wa[2], wa[3]);
+        if constexpr (kBFmt == 5) {
+          // rows 128a + 32c + lane, 16 B each (k-step j = word j) -> line (k-step j, atom a)
+          uint4 v[2][4];
+#pragma unroll
+          for (int a = 0; a < 2; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              v[a][c] = *reinterpret_cast<const uint4*>(sf + kSfBOff + 16 * (128 * a + 32 * c + lane));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+              const uint32_t w0 = j == 0 ? v[a][0].x : j == 1 ? v[a][0].y : j == 2 ? v[a][0].z : v[a][0].w;
+              const uint32_t w1 = j == 0 ? v[a][1].x : j == 1 ? v[a][1].y : j == 2 ? v[a][1].z : v[a][1].w;
+              const uint32_t w2 = j == 0 ? v[a][2].x : j == 1 ? v[a][2].y : j == 2 ? v[a][2].z : v[a][2].w;
+              const uint32_t w3 = j == 0 ? v[a][3].x : j == 1 ? v[a][3].y : j == 2 ? v[a][3].z : v[a][3].w;
+              *reinterpret_cast<uint4*>(sf + kSfBOff + 1024 * j + 512 * a + 16 * lane) =
+                  make_uint4(w0, w1, w2, w3);
+            }
+        } else {
+          // the two weight blocks' scales, the same for every row of their atom
+          const uint4 rg = *reinterpret_cast<const uint4*>(sf + kSfBRawE4);
+          const uint4 ru = *reinterpret_cast<const uint4*>(sf + kSfBRawE4 + 16);
+          const uint32_t xg[4] = {rg.x, rg.y, rg.z, rg.w}, xu[4] = {ru.x, ru.y, ru.z, ru.w};
+          uint32_t wb0 = 0, wb1 = 0;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nk) {
+              wb0 |= ((xg[j] >> 23) & 0xFFu) << (8 * j);
+              wb1 |= ((xu[j] >> 23) & 0xFFu) << (8 * j);
+              bad |= not_pow2_scale(xg[j]) | not_pow2_scale(xu[j]);
+            }
+          }
+          *reinterpret_cast<uint4*>(sf + kSfBOff + 16 * lane) = make_uint4(wb0, wb0, wb0, wb0);
+          *reinterpret_cast<uint4*>(sf + kSfBOff + 512 + 16 * lane) = make_uint4(wb1, wb1, wb1, wb1);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          if constexpr (kPair) mbar_arrive_cluster(full_lead0 + slot * sizeof(uint64_t));
+          else mbar_arrive(&ss.sf_full[slot]);
+        }
+      }
+      pipe.sf_it = g0 + static_cast<uint32_t>(n_grp);
+      // the k-steps the MMA issuer consumed in this phase: a later phase with the stager
+      // publishes ready counts in the issuer's own sequence
+      pipe.st_it += static_cast<uint32_t>(my_tiles * KB);
+      // the exponent fields were used all the same: the result is undefined, the call fails
+      if (bad) report_error(p.err, MOE_ERR_UNSUPPORTED, SITE_SCALE_FORMAT);
+    }
   } else if (warp >= 4) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant (the warp's 32 rows)
@@ -889,6 +1022,25 @@ __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtens
     pipe.tiles = tiles;
   }
 
+}
+
+// One grouped GEMM phase.  E2M1 weights need two scale copies every k-step on the MMA-issuing
+// thread; over a K loop of 8 or more k-steps the stager warp taking the stage-barrier waits
+// off that thread is measured faster.  E4M3 and BF16 kinds issue far fewer copies, and
+// shorter K loops do not amortise the hand-off: both lose more to it than they gain.  The
+// choice is per phase; the pipeline counters stay in step across phases of either kind.
+template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm = kBM>
+__device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
+                                           const TcParams& p, const Smem& sm, Pipe& pipe) {
+  if constexpr (kBlockScaled && kBFmt == 5) {
+    if (p.K >= 8 * 128) {
+      gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, true>(tmA_, tmB_, p, sm,
+                                                                             pipe);
+      return;
+    }
+  }
+  gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, false>(tmA_, tmB_, p, sm,
+                                                                          pipe);
 }
 
 }  // namespace gemm

@@ -25,6 +25,12 @@ EDGE = {
     "mixtral_bf16_one_expert": W_["mixtral_bf16"].scaled(T=70, H=256, E=1, k=1, I=256),
     "decode_fp8_fp4_T1": W_["decode_fp8_fp4"].scaled(T=1, H=512, E=16, k=8, I=256),
     "skewed_fp8_fp4_T1": W_["skewed_fp8_fp4"].scaled(T=1, H=256, E=64, k=16, I=128),
+    # E2M1 weights: the GEMM's stager warp runs for K loops of 8 or more 128-deep k-steps
+    # only, so in the persistent kernel one GEMM phase takes it and the other does not
+    "decode_fp8_fp4_short_then_long_k": W_["decode_fp8_fp4"].scaled(T=24, H=512, E=8, k=4,
+                                                                    I=1024),
+    "skewed_fp8_fp4_long_then_short_k": W_["skewed_fp8_fp4"].scaled(T=40, H=1024, E=16, k=4,
+                                                                    I=512),
 }
 
 
@@ -35,8 +41,13 @@ def _clean():
     M.moe_set_gemm_tiles("auto")
 
 
-@pytest.mark.parametrize("tiles", ["auto", "single", "small"])
-@pytest.mark.parametrize("name", list(EDGE))
+def _pair_cases():
+    return [(n, "pair") for n in EDGE if n.endswith("_k")]
+
+
+@pytest.mark.parametrize("name,tiles",
+                         [(n, t) for n in EDGE for t in ("auto", "single", "small")]
+                         + _pair_cases())
 def test_forward_matches_oracle(name, tiles):
     wl = EDGE[name]
     d = synth.make_inputs(wl, DEV)
