@@ -7,17 +7,20 @@
 namespace moe {
 namespace {
 
+constexpr int kRouteWarps = 8;
+
 template <int NPL>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(32 * kRouteWarps, 3) route_kernel(const float* __restrict__ logits,
                                                     const float* __restrict__ bias, int T, int E,
                                                     int k, int sigmoid, int renorm,
                                                     int32_t* __restrict__ topk_idx,
                                                     float* __restrict__ topk_w, int n_group,
                                                     int topk_group, float scale) {
-  const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  __shared__ __align__(8) uint8_t scratch[kRouteWarps][kRouteScratchBytes];
+  const int t = blockIdx.x * kRouteWarps + (threadIdx.x >> 5);
   if (t >= T) return;
   route_token<NPL>(logits, bias, t, E, k, sigmoid, renorm, topk_idx, topk_w, threadIdx.x & 31,
-                   n_group, topk_group, scale);
+                   scratch[threadIdx.x >> 5], n_group, topk_group, scale);
 }
 
 }  // namespace
@@ -25,8 +28,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 cudaError_t launch_route(const float* logits, const float* bias, int T, int E, int k, int score,
                          int renorm, int32_t* topk_idx, float* topk_w, cudaStream_t s,
                          int n_group, int topk_group, float scale) {
-  const int warps = 8;
-  dim3 grid((T + warps - 1) / warps), block(32 * warps);
+  dim3 grid((T + kRouteWarps - 1) / kRouteWarps), block(32 * kRouteWarps);
   const int sig = score == MOE_SCORE_SIGMOID;
   const int npl = (E + 31) / 32;
   count_launch();

@@ -47,13 +47,27 @@ __device__ __forceinline__ float sigmoid_keys_f32(float l) {
   return __fdiv_rn(1.0f, __fadd_rn(1.0f, exp_keys_f32(-l)));
 }
 
-// (key, id) ordering: larger key first, then lower id.
-__device__ __forceinline__ bool better(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
+// Order-preserving integer of an fp32 selection key (-0 taken as +0, so that equal keys give
+// equal words; NaNs order by their bit patterns).
+__device__ __forceinline__ uint32_t ord_key(float key) {
+  const uint32_t u = __float_as_uint(__fadd_rn(key, 0.0f));
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// A candidate as one 64-bit word ordered like (key, id): the ordered key in the high half, the
+// complemented id in the low half (lower id wins a tie).  0 is below every candidate.
+__device__ __forceinline__ uint64_t pack_cand(uint32_t ku, int e) {
+  return (static_cast<uint64_t>(ku) << 32) | static_cast<uint32_t>(~e);
+}
+
+// Per-warp shared-memory scratch of route_token: kRouteCand packed candidates, then the k
+// selected ids.
+constexpr int kRouteCand = 128;
+constexpr int kRouteScratchBytes = kRouteCand * 8 + 32 * 4;
+
 // One warp selects the k experts of token t and writes topk_idx[t, :], topk_w[t, :].
-// Lanes hold experts lane, lane+32, ...; all 32 lanes must call it together.
+// Lanes hold experts lane, lane+32, ...; all 32 lanes must call it together, each warp with
+// its own kRouteScratchBytes of 8-byte aligned shared memory.
 // Group-limited selection (n_group > 1, groups of G = E / n_group experts with G a multiple
 // of 32): a group's score is the fp32 sum of its two largest keys, the topk_group best groups
 // (equal scores -> lower group) are kept and the k experts are chosen among theirs only.
@@ -65,46 +79,26 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
                                             int sigmoid, int renorm,
                                             int32_t* __restrict__ topk_idx,
                                             float* __restrict__ topk_w, int lane,
-                                            int n_group = 1, int topk_group = 1,
-                                            float scale = 1.0f) {
+                                            uint8_t* scratch, int n_group = 1,
+                                            int topk_group = 1, float scale = 1.0f) {
   const float* row = logits + static_cast<size_t>(t) * E;
 
   float key[NPL];
-  float val[NPL];  // softmax: the logit; sigmoid: s
 #pragma unroll
   for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
       const float l = __ldg(row + e);
-      if (sigmoid) {
-        const float s = sigmoid_keys_f32(l);
-        val[i] = s;
-        key[i] = __fadd_rn(s, bias ? __ldg(bias + e) : 0.0f);
-      } else {
-        val[i] = l;
-        key[i] = l;
-      }
+      key[i] = sigmoid ? __fadd_rn(sigmoid_keys_f32(l), bias ? __ldg(bias + e) : 0.0f) : l;
     } else {
-      val[i] = 0.0f;
       key[i] = -INFINITY;
     }
   }
 
-  // Selection.  A candidate is packed into one 64-bit word ordered like (key, id): the key
-  // as an order-preserving integer in the high half (-0 taken as +0, so that equal keys give
-  // equal words), the complemented id in the low half (lower id wins a tie).  0 is below
-  // every candidate.  Each lane caches its best four untaken candidates; a round takes the
-  // warp maximum of the lanes' best (5 shuffle steps), the winning lane moves its list up,
-  // and only a lane whose four are all taken rescans its NPL experts.
-  auto pack = [](float key, int e) -> uint64_t {
-    uint32_t u = __float_as_uint(__fadd_rn(key, 0.0f));
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    return (static_cast<uint64_t>(u) << 32) | static_cast<uint32_t>(~e);
-  };
   // Groups.  Lane l holds experts l + 32i, so with G a multiple of 32 a group is sg = G / 32
   // consecutive slots i of every lane: each lane keeps a running top-2 over the group's
   // slots and the warp merges them at the group's last slot; slots of groups that are not
-  // kept start out as taken.
+  // kept are not candidates.
   uint32_t taken = 0;
   if (n_group > 1) {
     const int sg = E / n_group / 32;
@@ -151,87 +145,136 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
       if (!((keep >> last) & 1u)) taken |= 1u << i;
     }
   }
-  // This lane's best four untaken candidates in order (c[0] best; 0 = none) and their
-  // values; the winning lane shifts its list up and rescans only once all four are gone.
-  constexpr int kC = 4;
-  uint64_t c[kC];
-  float cv[kC];
-  int n_c = 0;  // valid entries of c
-  auto scan = [&]() {
+
+  // Ordered keys of this lane's eligible experts (0 marks an ineligible slot; the ordered
+  // key of an eligible one may be 0 too, which only ever adds candidates below).
+  uint32_t elig = 0;
+  uint32_t ku[NPL];
+  uint32_t m = 0;  // this lane's largest ordered key
 #pragma unroll
-    for (int q = 0; q < kC; ++q) {
-      c[q] = 0;
-      cv[q] = 0.0f;
+  for (int i = 0; i < NPL; ++i) {
+    const bool ok = lane + 32 * i < E && !((taken >> i) & 1u);
+    ku[i] = ok ? ord_key(key[i]) : 0u;
+    elig |= static_cast<uint32_t>(ok) << i;
+    m = max(m, ku[i]);
+  }
+
+  // Selection.  A lower bound of the k-th best key: the k-th largest of the 32 lane maxima
+  // (bitonic sort of the lane maxima across the warp).  When it is above 0, k lanes hold a
+  // key at or above it, so every one of the k best is a key at or above it; at 0 every
+  // eligible expert is a candidate.  The candidates (a few dozen on router logits) are
+  // compacted into shared memory in (slot, lane) order and each is ranked by the number of
+  // candidates above it in (key, id) order, which is exact and has no ties (ids differ).
+  uint32_t v = m;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const uint32_t o = __shfl_xor_sync(0xffffffffu, v, stride);
+      const bool lower = (lane & stride) == 0, up = (lane & size) == 0;
+      v = (lower == up) ? min(v, o) : max(v, o);
     }
+  }
+  const uint32_t bound = __shfl_sync(0xffffffffu, v, 32 - k);  // ascending across lanes
+
+  uint64_t* cand = reinterpret_cast<uint64_t*>(scratch);
+  int32_t* sel = reinterpret_cast<int32_t*>(scratch + kRouteCand * 8);
+  const uint32_t below = (1u << lane) - 1u;
+  int n = 0;  // candidates so far (warp-uniform)
 #pragma unroll
-    for (int i = 0; i < NPL; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !((taken >> i) & 1u)) {
-        const uint64_t x = pack(key[i], e);
-        if (x > c[kC - 1]) {  // insert, keeping c sorted
-          uint64_t y = x;
-          float yv = val[i];
+  for (int i = 0; i < NPL; ++i) {
+    const bool is_c = ((elig >> i) & 1u) && ku[i] >= bound;
+    const uint32_t bal = __ballot_sync(0xffffffffu, is_c);
+    if (is_c) {
+      const int pos = n + __popc(bal & below);
+      if (pos < kRouteCand) cand[pos] = pack_cand(ku[i], lane + 32 * i);
+    }
+    n += __popc(bal);
+  }
+  __syncwarp();
+
+  int my_idx = 0;  // lane j keeps the j-th selection
+  if (n <= kRouteCand) {
+    for (int j = lane; j < n; j += 32) {
+      const uint64_t cj = cand[j];
+      int r = 0;
+#pragma unroll 4
+      for (int i = 0; i < n; ++i) r += cand[i] > cj;
+      if (r < k) sel[r] = static_cast<int>(~static_cast<uint32_t>(cj));
+    }
+    __syncwarp();
+    if (lane < k) my_idx = sel[lane];
+  } else {
+    // Many keys tie at the bound (constant logits, say): k rounds of a warp maximum over
+    // each lane's best four untaken candidates; the winning lane moves its list up and
+    // rescans its NPL experts only once all four are taken.
+    constexpr int kC = 4;
+    uint64_t c[kC];
+    int n_c = 0;  // valid entries of c
+    auto scan = [&]() {
 #pragma unroll
-          for (int q = 0; q < kC; ++q) {
-            if (y > c[q]) {
-              const uint64_t t0 = c[q];
-              const float tv = cv[q];
-              c[q] = y;
-              cv[q] = yv;
-              y = t0;
-              yv = tv;
+      for (int q = 0; q < kC; ++q) c[q] = 0;
+#pragma unroll
+      for (int i = 0; i < NPL; ++i) {
+        if ((elig >> i) & 1u) {
+          uint64_t y = pack_cand(ku[i], lane + 32 * i);
+          if (y > c[kC - 1]) {  // insert, keeping c sorted
+#pragma unroll
+            for (int q = 0; q < kC; ++q) {
+              if (y > c[q]) {
+                const uint64_t t0 = c[q];
+                c[q] = y;
+                y = t0;
+              }
             }
           }
         }
       }
-    }
-    n_c = 0;
+      n_c = 0;
 #pragma unroll
-    for (int q = 0; q < kC; ++q) n_c += c[q] != 0;
-  };
-  scan();
-  int my_idx = 0;      // lane j keeps the j-th selection
-  float my_val = 0.0f;
-  float top_val = 0.0f;
-  for (int j = 0; j < k; ++j) {
-    uint64_t best = c[0];
+      for (int q = 0; q < kC; ++q) n_c += c[q] != 0;
+    };
+    scan();
+    for (int j = 0; j < k; ++j) {
+      uint64_t best = c[0];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
-      best = o > best ? o : best;
-    }
-    const int bi = static_cast<int>(~static_cast<uint32_t>(best));
-    const int owner = bi & 31;
-    const float bv = __shfl_sync(0xffffffffu, cv[0], owner);
-    if (lane == owner) {
-      taken |= 1u << (bi >> 5);
-      if (n_c > 1) {
-#pragma unroll
-        for (int q = 0; q + 1 < kC; ++q) {
-          c[q] = c[q + 1];
-          cv[q] = cv[q + 1];
-        }
-        c[kC - 1] = 0;
-        --n_c;
-      } else {
-        scan();
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+        best = o > best ? o : best;
       }
+      const int bi = static_cast<int>(~static_cast<uint32_t>(best));
+      if (lane == (bi & 31)) {
+        elig &= ~(1u << (bi >> 5));
+        if (n_c > 1) {
+#pragma unroll
+          for (int q = 0; q + 1 < kC; ++q) c[q] = c[q + 1];
+          c[kC - 1] = 0;
+          --n_c;
+        } else {
+          scan();
+        }
+      }
+      if (lane == j) my_idx = bi;
     }
-    if (lane == j) {
-      my_idx = bi;
-      my_val = bv;
-    }
-    if (j == 0) top_val = bv;
   }
+  __syncwarp();  // the scratch is free for the next token
+
+  // The selected experts' values, recomputed from their logits exactly as the keys were
+  // (softmax: the logit; sigmoid: s).
+  float my_val = 0.0f;
+  if (lane < k) {
+    const float l = __ldg(row + my_idx);
+    my_val = sigmoid ? sigmoid_keys_f32(l) : l;
+  }
+  const float top_val = __shfl_sync(0xffffffffu, my_val, 0);
 
   float g;
   if (sigmoid) {
     g = (lane < k) ? my_val : 0.0f;
     if (renorm) {
-      float sum = g;
       // rank-order sum: lanes 0..k-1 hold the selected s in rank order
       float acc = 0.0f;
-      for (int j = 0; j < k; ++j) acc += __shfl_sync(0xffffffffu, sum, j);
+      for (int j = 0; j < k; ++j) acc += __shfl_sync(0xffffffffu, g, j);
       g = g / acc;
     }
   } else {
@@ -243,7 +286,7 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
       float part = 0.0f;
 #pragma unroll
       for (int i = 0; i < NPL; ++i)
-        if (lane + 32 * i < E) part += expf(val[i] - top_val);
+        if (lane + 32 * i < E) part += expf(__ldg(row + lane + 32 * i) - top_val);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
       den = part;

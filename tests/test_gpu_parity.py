@@ -89,6 +89,30 @@ def test_route_edges(score, T, E, k):
         assert np.max(np.abs(w.cpu().numpy() - rw) / np.maximum(rw, 1e-30)) < 2e-6
 
 
+@pytest.mark.parametrize("score", ["softmax", "sigmoid"])
+@pytest.mark.parametrize("E,k", [(256, 8), (1024, 16), (1024, 32), (100, 5)])
+def test_route_tied_keys(score, E, k):
+    """Keys that tie at and around the k-th best: logits on a coarse grid (a few dozen to
+    hundreds of equal keys per row), +0 / -0 mixes and -inf logits.  The router's selection
+    takes its exact candidate ranking when few keys reach its bound and its fallback when
+    many do; both must give the oracle's (key desc, id asc) order."""
+    g = torch.Generator(device=DEV).manual_seed(E * 7 + k)
+    T = 96
+    logits = torch.round(torch.randn((T, E), generator=g, device=DEV) * 2.0) / 2.0
+    logits[1::3] = torch.round(torch.randn((T // 3, E), generator=g, device=DEV) * 0.3)
+    zeros = torch.zeros(E, device=DEV)
+    zeros[torch.arange(0, E, 2, device=DEV)] = -0.0
+    logits[2] = zeros                                         # +0 / -0 only
+    logits[5, torch.arange(0, E, 3, device=DEV)] = float("-inf")
+    bias = torch.randn(E, generator=g, device=DEV) * 0.1 if score == "sigmoid" else None
+    for renorm in (True, False):
+        idx, w = M.moe_route(logits, k, score, bias=bias, renorm=renorm)
+        ridx, rw = oracle.route(logits.cpu().numpy(),
+                                None if bias is None else bias.cpu().numpy(), k, score, renorm)
+        assert np.array_equal(idx.cpu().numpy(), ridx)
+        assert np.max(np.abs(w.cpu().numpy() - rw) / np.maximum(rw, 1e-30)) < 2e-6
+
+
 # ------------------------------------------------------------------------------- dispatch
 def _check_dispatch(wl, d, idx):
     r = M.moe_dispatch(d["x"], idx, wl.E, wl.act, x_scales=d["x_scales"])
