@@ -38,7 +38,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # smaller case with the same rows per expert (dram__bytes_read.sum + dram__bytes_write.sum
 # of one launch).  Used for the roofline's "traffic".
 TRAFFIC_RATIO = {
-    ("v3_fp8", "linear1"): (1.151, "the V3-shaped layer at T=1024, E=32"),
+    ("v3_fp8", "linear1"): (1.153, "the V3-shaped layer at T=1024, E=32"),
+    ("v3_fp8", "linear2"): (0.972, "the V3-shaped layer at T=1024, E=32"),
+    ("decode_fp8_fp4", "linear1"): (1.013, "the decode-shaped layer at E=64"),
 }
 
 
@@ -414,6 +416,11 @@ def run_native(args, ws, rank, local):
         "scale_fmt": args.scale_fmt,
         "chain_ms_per_step": chain_ms,
         "stage_ms": stage_ms,
+        # algorithmic bytes of each stage over its CUDA-event time, and that over the
+        # measured copy bandwidth (the memory-bound stages' roofline)
+        "stage_gbps": {n: alg[n]["bytes"] / (stage_ms[n] / 1e3) / 1e9 for n in names},
+        "stage_hbm_frac": {n: alg[n]["bytes"] / (stage_ms[n] / 1e3) / 1e9 / pk["hbm_gbs"]
+                           for n in names},
         "roofline": roof,
         "e2e": {"value": T * ws / (e2e_ms / 1e3), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -574,6 +581,58 @@ def run_reference(args, ws, rank):
     }
 
 
+def run_route(args, ws, rank, local):
+    """The router alone on the workload's logits (profiling captures of route_kernel at the
+    full token count without the expert weights on the device)."""
+    import moe_expert_layer_prefix_b200 as M
+
+    wl = workload(args)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d = synth.make_activations(wl, dev)
+    idx = torch.empty((wl.T, wl.k), dtype=torch.int32, device=dev)
+    gw = torch.empty((wl.T, wl.k), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        M.moe_route(d["logits"], wl.k, wl.score, bias=d["bias"], renorm=wl.renorm,
+                    topk_idx=idx, topk_w=gw, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    clocks = Clocks(local)
+    clocks.start()
+    time.sleep(0.3)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws) / args.steps
+    clk = clocks.stop()
+    st, site = M.moe_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {M.moe_status_string(st)} at site {site}")
+    pk, pk_kind = peaks()
+    byt = algorithmic(wl, wl.E)["route"]["bytes"]
+    return {
+        "metric": "router tokens/s (moe_route alone)", "value": wl.T * ws / (ms / 1e3),
+        "unit": "tokens/s", "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32", "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "T": wl.T, "E": wl.E, "k": wl.k,
+                   "router": wl.score, "logits": wl.logits},
+        "roofline": {"bound": "hbm", "achieved": byt / (ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "frac": byt / (ms / 1e3) / 1e9 / pk["hbm_gbs"],
+                     "peak_note": f"{pk_kind} copy bandwidth", "kernel": "route"},
+        "clocks": clk,
+    }
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -583,6 +642,8 @@ def main():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--bf16-input", action="store_true",
                     help="E4M3 workloads: feed BF16 activations, quantised in the dispatch")
+    ap.add_argument("--route-only", action="store_true",
+                    help="time the router alone on the workload's logits")
     ap.add_argument("--backward", action="store_true",
                     help="time the BF16 layer's backward (moe_expert_backward) instead")
     ap.add_argument("--scale-fmt", default="pow2", choices=["pow2", "fp32"],
@@ -603,6 +664,8 @@ def main():
     ws, rank, local = dist_setup(args)
     if args.impl == "reference":
         res = run_reference(args, ws, rank) if rank == 0 else None
+    elif args.route_only:
+        res = run_route(args, ws, rank, local)
     elif args.backward:
         res = run_backward(args, ws, rank, local)
     else:

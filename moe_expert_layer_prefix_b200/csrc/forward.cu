@@ -88,15 +88,12 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   do {
     // 1. route: one warp per token, candidate scratch per warp in the idle GEMM ring
     uint8_t* rscr = scratch + warp * kRouteScratchBytes;
-    if (p.E <= 256) {
-      for (int t = gw; t < p.T; t += GW)
-        route_token<8>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
-                       rscr, p.n_group, p.topk_group, p.scale);
-    } else {
-      for (int t = gw; t < p.T; t += GW)
-        route_token<32>(p.logits, p.bias, t, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx, p.topk_w, lane,
-                        rscr, p.n_group, p.topk_group, p.scale);
-    }
+    if (p.E <= 256)
+      route_tokens<8>(p.logits, p.bias, gw, GW, p.T, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx,
+                      p.topk_w, lane, rscr, p.n_group, p.topk_group, p.scale);
+    else
+      route_tokens<32>(p.logits, p.bias, gw, GW, p.T, p.E, p.k, p.sigmoid, p.renorm, p.topk_idx,
+                       p.topk_w, lane, rscr, p.n_group, p.topk_group, p.scale);
     if (!grid_sync(p.bar, p.err)) break;
 
     // 2. per-chunk expert counts

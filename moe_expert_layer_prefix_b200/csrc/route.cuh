@@ -73,14 +73,27 @@ constexpr int kRouteScratchBytes = kRouteCand * 8 + 32 * 4;
 // (equal scores -> lower group) are kept and the k experts are chosen among theirs only.
 // Gates are multiplied by `scale` (the routed scaling factor).  n_group = 1, scale = 1 is
 // the plain router.
+// Token t's logits, lane l holding experts l, l + 32, ... (0 past E).
+template <int NPL>
+__device__ __forceinline__ void route_load(const float* __restrict__ logits, int t, int E,
+                                           int lane, float (&l)[NPL]) {
+  const float* row = logits + static_cast<size_t>(t) * E;
+#pragma unroll
+  for (int i = 0; i < NPL; ++i) {
+    const int e = lane + 32 * i;
+    l[i] = e < E ? __ldg(row + e) : 0.0f;
+  }
+}
+
 template <int NPL>  // experts per lane (E <= 32 * NPL)
-__device__ __forceinline__ void route_token(const float* __restrict__ logits,
-                                            const float* __restrict__ bias, int t, int E, int k,
-                                            int sigmoid, int renorm,
-                                            int32_t* __restrict__ topk_idx,
-                                            float* __restrict__ topk_w, int lane,
-                                            uint8_t* scratch, int n_group = 1,
-                                            int topk_group = 1, float scale = 1.0f) {
+__device__ __forceinline__ void route_select(const float (&lg)[NPL],
+                                             const float* __restrict__ logits,
+                                             const float* __restrict__ bias, int t, int E, int k,
+                                             int sigmoid, int renorm,
+                                             int32_t* __restrict__ topk_idx,
+                                             float* __restrict__ topk_w, int lane,
+                                             uint8_t* scratch, int n_group, int topk_group,
+                                             float scale) {
   const float* row = logits + static_cast<size_t>(t) * E;
 
   float key[NPL];
@@ -88,7 +101,7 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
   for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
     if (e < E) {
-      const float l = __ldg(row + e);
+      const float l = lg[i];
       key[i] = sigmoid ? __fadd_rn(sigmoid_keys_f32(l), bias ? __ldg(bias + e) : 0.0f) : l;
     } else {
       key[i] = -INFINITY;
@@ -296,6 +309,44 @@ __device__ __forceinline__ void route_token(const float* __restrict__ logits,
   if (lane < k) {
     topk_idx[static_cast<size_t>(t) * k + lane] = my_idx;
     topk_w[static_cast<size_t>(t) * k + lane] = g * scale;
+  }
+}
+
+// One token: its logits, then its selection.
+template <int NPL>
+__device__ __forceinline__ void route_token(const float* __restrict__ logits,
+                                            const float* __restrict__ bias, int t, int E, int k,
+                                            int sigmoid, int renorm,
+                                            int32_t* __restrict__ topk_idx,
+                                            float* __restrict__ topk_w, int lane,
+                                            uint8_t* scratch, int n_group = 1,
+                                            int topk_group = 1, float scale = 1.0f) {
+  float l[NPL];
+  route_load<NPL>(logits, t, E, lane, l);
+  route_select<NPL>(l, logits, bias, t, E, k, sigmoid, renorm, topk_idx, topk_w, lane, scratch,
+                    n_group, topk_group, scale);
+}
+
+// Tokens t0, t0 + stride, ... by one warp, the next token's logits loaded while the current
+// one is selected (a warp that walks several tokens would otherwise wait out each load).
+template <int NPL>
+__device__ __forceinline__ void route_tokens(const float* __restrict__ logits,
+                                             const float* __restrict__ bias, int t0, int stride,
+                                             int T, int E, int k, int sigmoid, int renorm,
+                                             int32_t* __restrict__ topk_idx,
+                                             float* __restrict__ topk_w, int lane,
+                                             uint8_t* scratch, int n_group, int topk_group,
+                                             float scale) {
+  if (t0 >= T) return;
+  float nxt[NPL];
+  route_load<NPL>(logits, t0, E, lane, nxt);
+  for (int t = t0; t < T; t += stride) {
+    float cur[NPL];
+#pragma unroll
+    for (int i = 0; i < NPL; ++i) cur[i] = nxt[i];
+    if (t + stride < T) route_load<NPL>(logits, t + stride, E, lane, nxt);
+    route_select<NPL>(cur, logits, bias, t, E, k, sigmoid, renorm, topk_idx, topk_w, lane,
+                      scratch, n_group, topk_group, scale);
   }
 }
 
