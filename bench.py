@@ -381,7 +381,9 @@ def run_native(args, ws, rank, local):
     roof["kernel"] = dom
     if args.traffic is not None:
         roof["traffic"] = args.traffic
-    elif (wl.name, dom) in TRAFFIC_RATIO:
+    elif (wl.name, dom) in TRAFFIC_RATIO and args.scale_fmt == "pow2" and args.tiles == "auto":
+        # (the ratios were measured on the power-of-two-scale kernels at the automatic tile
+        # shape; other paths run other kernels)
         ratio, src = TRAFFIC_RATIO[(wl.name, dom)]
         roof["traffic"] = ratio * alg[dom]["bytes"]
         roof["traffic_note"] = (f"DRAM read+write bytes per launch = {ratio} x algorithmic, "
