@@ -137,6 +137,7 @@ template <int kCta, int kTm = kBM>
 struct Cfg {
   static_assert(kTm == kBM || (kCta == 1 && kTm == 32), "unsupported tile shape");
   static constexpr int kStages = kCta == 2 ? 6 : (kTm == kBM ? 4 : 5);
+  static_assert(kStages <= kMaxStages, "the stage barriers would overlap the next ones");
   static constexpr int kATileBytes = kTm * kRowBytes;     // 16 KB (4 KB small)
   static constexpr int kBRows = kBN / kCta;               // B rows this CTA loads per k-step
   static constexpr int kBTileBytes = kBRows * kRowBytes;  // 32 KB single, 16 KB pair
