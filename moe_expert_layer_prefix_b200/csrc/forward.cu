@@ -55,14 +55,16 @@ struct FwdParams {
   TcParams l1, l2;
 };
 
-template <bool kBS, int kBFmt, bool kE4, int kTm>
+// kCta = 2: the GEMM phases run on CTA pairs (cta_group::2, M = 256 tiles); the launch is
+// then a cluster launch of pairs, and every other phase treats the CTAs as before.
+template <bool kBS, int kBFmt, bool kE4, int kTm, int kCta>
 __global__ void __launch_bounds__(kThreads, 1)
 moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW1,
                    const __grid_constant__ CUtensorMap tmH, const __grid_constant__ CUtensorMap tmW2,
                    const FwdParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const Smem sm = carve<1, kTm>(smem_raw);
-  gemm_init<1, kBS, kTm>(sm, &tmX, 1);
+  const Smem sm = carve<kCta, kTm>(smem_raw);
+  gemm_init<kCta, kBS, kTm>(sm, &tmX, 1);
   if (threadIdx.x == 0) {
     tma_prefetch_desc(&tmW1);
     tma_prefetch_desc(&tmH);
@@ -70,6 +72,7 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
   }
   tc_fence_before();
   __syncthreads();
+  if constexpr (kCta == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -132,16 +135,16 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
     // 7. linear-1 + SwiGLU + requantisation.  The m-block list is computed once for both
     //    GEMMs (the same offsets and tile shape).
     Pipe pipe;
-    gemm_prefix<1, kTm>(sm, p.offsets, p.E);
+    gemm_prefix<kCta, kTm>(sm, p.offsets, p.E);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    gemm_phase<1, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
+    gemm_phase<kCta, kBS, kBFmt, true, kE4, kTm>(&tmX, &tmW1, p.l1, sm, pipe);
     fence_proxy_async_global();  // h is read by TMA next
     if (!grid_sync(p.bar, p.err)) break;
 
     // 8. linear-2
-    gemm_phase<1, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
+    gemm_phase<kCta, kBS, kBFmt, false, false, kTm>(&tmH, &tmW2, p.l2, sm, pipe);
     if (!grid_sync(p.bar, p.err)) break;
 
     // 9. combine.  A warp keeps two 16-byte loads per lane and source row in flight and
@@ -164,11 +167,13 @@ moe_forward_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constan
 
   tc_fence_before();
   __syncthreads();
+  // in a pair, neither CTA leaves while the other may still touch its shared memory
+  if constexpr (kCta == 2) cluster_sync();
   tc_fence_after();
-  gemm_fini<1>(sm);
+  gemm_fini<kCta>(sm);
 }
 
-template <bool kBS, int kBFmt, bool kE4, int kTm>
+template <bool kBS, int kBFmt, bool kE4, int kTm, int kCta>
 cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   const int S = a.T * a.k;
   const int afmt = a.act == MOE_BF16 ? 0 : 1;
@@ -234,23 +239,41 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
   p.l1 = l1;
   p.l2 = l2;
 
-  auto kern = moe_forward_kernel<kBS, kBFmt, kE4, kTm>;
-  const size_t smem = Cfg<1, kTm>::kSmem;
+  auto kern = moe_forward_kernel<kBS, kBFmt, kE4, kTm, kCta>;
+  const size_t smem = Cfg<kCta, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
-  if (err != cudaSuccess) return err;
-  err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), s);
   if (err != cudaSuccess) return err;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms());
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
+  if constexpr (kCta == 2) {
+    // pairs: as many clusters as can be resident at once (every CTA waits at the grid
+    // barriers, so all of them must be), at most one CTA per SM
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t q = cfg;
+    q.attrs = attr + 1;
+    q.numAttrs = 1;
+    int clusters = 0;
+    err = cudaOccupancyMaxActiveClusters(&clusters, kern, &q);
+    if (err != cudaSuccess) return err;
+    clusters = min(clusters, num_sms() / 2);
+    if (clusters < 1) return cudaErrorNotSupported;
+    cfg.gridDim = dim3(2 * clusters);
+    cfg.numAttrs = 2;
+  }
+  err = cudaMemsetAsync(a.bar, 0, 2 * sizeof(uint32_t), s);
+  if (err != cudaSuccess) return err;
   count_launch();
   return cudaLaunchKernelEx(&cfg, kern, tmX, tmW1, tmH, tmW2, p);
 }
@@ -260,13 +283,20 @@ cudaError_t launch(const ForwardArgs& a, cudaStream_t s) {
 cudaError_t launch_forward_fused(const ForwardArgs& a, cudaStream_t s) {
   // the dispatch phases keep per-warp masks (8 x E words) in the idle GEMM ring
   if (a.E > 1024) return cudaErrorNotSupported;
-  const bool small = gemm_tile_shape(a.act, a.T * a.k, a.E, false) == 3;
+  // the chain's tile choice (1 single, 2 pair, 3 small), so that both compute the same bytes
+  const int shape = gemm_tile_shape(a.act, a.T * a.k, a.E, true);
   if (a.act == MOE_BF16 && a.wt == MOE_BF16)
-    return small ? launch<false, 0, false, 32>(a, s) : launch<false, 0, false, kBM>(a, s);
+    return shape == 3   ? launch<false, 0, false, 32, 1>(a, s)
+           : shape == 2 ? launch<false, 0, false, kBM, 2>(a, s)
+                        : launch<false, 0, false, kBM, 1>(a, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E4M3)
-    return small ? launch<true, 0, true, 32>(a, s) : launch<true, 0, true, kBM>(a, s);
+    return shape == 3   ? launch<true, 0, true, 32, 1>(a, s)
+           : shape == 2 ? launch<true, 0, true, kBM, 2>(a, s)
+                        : launch<true, 0, true, kBM, 1>(a, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E2M1)
-    return small ? launch<true, 5, true, 32>(a, s) : launch<true, 5, true, kBM>(a, s);
+    return shape == 3   ? launch<true, 5, true, 32, 1>(a, s)
+           : shape == 2 ? launch<true, 5, true, kBM, 2>(a, s)
+                        : launch<true, 5, true, kBM, 1>(a, s);
   return cudaErrorNotSupported;
 }
 

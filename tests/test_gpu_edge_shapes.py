@@ -41,13 +41,8 @@ def _clean():
     M.moe_set_gemm_tiles("auto")
 
 
-def _pair_cases():
-    return [(n, "pair") for n in EDGE if n.endswith("_k")]
-
-
 @pytest.mark.parametrize("name,tiles",
-                         [(n, t) for n in EDGE for t in ("auto", "single", "small")]
-                         + _pair_cases())
+                         [(n, t) for n in EDGE for t in ("auto", "single", "small", "pair")])
 def test_forward_matches_oracle(name, tiles):
     wl = EDGE[name]
     d = synth.make_inputs(wl, DEV)
@@ -64,7 +59,7 @@ def test_forward_matches_oracle(name, tiles):
     assert_parity(host_values(out, None, fmt), r["out"], fmt, TOL[wl.act])
 
 
-@pytest.mark.parametrize("tiles", ["single", "small"])
+@pytest.mark.parametrize("tiles", ["single", "small", "pair"])
 @pytest.mark.parametrize("name", list(EDGE))
 def test_forward_equals_unfused_chain(name, tiles):
     wl = EDGE[name]
