@@ -284,9 +284,11 @@ typedef struct moe_backward_args {
  * Steps, each stored where the comment says:
  *   combine backward:  dy_w[slot] = BF16(w * dout[t]);  dgate = dout[t] . y[slot] (fp32)
  *   router backward:   dlogits (fp32) through the gate function
- *   G  = BF16(x_perm W1^T)  (pre-activations recomputed on the expert GEMM)
  *   dh = BF16(dy_w W2)       (expert GEMM on W2^T)
- *   dG = BF16(SwiGLU backward of G, dh)
+ *   dG = BF16(SwiGLU backward of (g, u), dh): the expert GEMM of linear-1 recomputes the
+ *        pre-activations (g, u) = x_perm W1^T in fp32 and its epilogue turns them and dh
+ *        into dg = dh u s (1 + g (1 - s)) and du = dh g s, s = sigmoid(g); g and u are
+ *        not stored
  *   dx_slot = BF16(dG W1)    (expert GEMM on W1^T);  dx[t] = BF16(sum of its k slots)
  *   dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e  (fp32; tensor cores, on copies of the
  *                                               operands transposed so that each expert's

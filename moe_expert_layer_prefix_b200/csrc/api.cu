@@ -177,7 +177,7 @@ size_t moe_workspace_size(int op, int T, int H, int E, int k, int I, int act, in
       if (act != MOE_BF16 || wt != MOE_BF16) return 0;
       size_t b = 0;
       b += round256(static_cast<size_t>(S) * H * 2) * 2;      // dy_w, dx_slot
-      b += round256(static_cast<size_t>(S) * 2 * I * 2) * 2;  // G, dG
+      b += round256(static_cast<size_t>(S) * 2 * I * 2);      // dG
       b += round256(static_cast<size_t>(S) * I * 2);          // dh
       b += round256(static_cast<size_t>(S) * 4) * 2;          // dgates, unit weights
       b += round256(static_cast<size_t>(E + 1) * 4);          // padded segment starts
@@ -528,7 +528,6 @@ moe_status moe_expert_backward(const moe_backward_args* a, void* ws, size_t ws_b
   };
   void* dy_w = take(static_cast<size_t>(S) * H * 2);
   void* dx_slot = take(static_cast<size_t>(S) * H * 2);
-  void* G = take(static_cast<size_t>(S) * 2 * I * 2);
   void* dG = take(static_cast<size_t>(S) * 2 * I * 2);
   void* dh = take(static_cast<size_t>(S) * I * 2);
   float* dgates = static_cast<float*>(take(static_cast<size_t>(S) * 4));
@@ -546,14 +545,15 @@ moe_status moe_expert_backward(const moe_backward_args* a, void* ws, size_t ws_b
                            stream) != cudaSuccess)
     return MOE_ERR_CUDA;
   // expert GEMM of the forward pass, out[S, N] = A[S, K] . W[E, N, K]^T: FfnArgs with
-  // I = K and H = N (its linear-2 form)
-  const FfnArgs g_args{MOE_BF16, MOE_BF16, a->x_perm, nullptr, a->expert_offsets, S, 2 * I, H,
-                       E, a->w1, nullptr, G, nullptr, err};
-  if (launch_linear2_tc(g_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  // I = K and H = N (its linear-2 form).  dh = dy_w . W2 first; then linear-1 in its backward
+  // form recomputes the pre-activations and turns them and dh into dG in its epilogue
   const FfnArgs dh_args{MOE_BF16, MOE_BF16, dy_w, nullptr, a->expert_offsets, S, I, H,
                         E, a->w2_t, nullptr, dh, nullptr, err};
   if (launch_linear2_tc(dh_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
-  if (launch_swiglu_backward(G, dh, S, I, dG, stream) != cudaSuccess) return MOE_ERR_CUDA;
+  FfnArgs dg_args{MOE_BF16, MOE_BF16, a->x_perm, nullptr, a->expert_offsets, S, H, I,
+                  E, a->w1, nullptr, dG, nullptr, err};
+  dg_args.dh = dh;
+  if (launch_linear1_dgate_tc(dg_args, stream) != cudaSuccess) return MOE_ERR_CUDA;
   const FfnArgs dx_args{MOE_BF16, MOE_BF16, dG, nullptr, a->expert_offsets, S, H, 2 * I,
                         E, a->w1_t, nullptr, dx_slot, nullptr, err};
   if (launch_linear2_tc(dx_args, stream) != cudaSuccess) return MOE_ERR_CUDA;

@@ -149,40 +149,6 @@ __global__ void __launch_bounds__(256) gate_backward_kernel(
 
 // dG = [dg | du] from the recomputed pre-activations G = [g | u] [S, 2I] and dh [S, I], in
 // fp32, stored BF16; 8 columns per thread.
-__global__ void __launch_bounds__(256) swiglu_backward_kernel(const __nv_bfloat16* __restrict__ G,
-                                                              const __nv_bfloat16* __restrict__ dh,
-                                                              int S, int I,
-                                                              __nv_bfloat16* __restrict__ dG) {
-  const int vpr = I / 8;
-  const long n_items = static_cast<long>(S) * vpr;
-  for (long it = static_cast<long>(blockIdx.x) * blockDim.x + threadIdx.x; it < n_items;
-       it += static_cast<long>(gridDim.x) * blockDim.x) {
-    const long n = it / vpr;
-    const int c = static_cast<int>(it % vpr) * 8;
-    const size_t grow = static_cast<size_t>(n) * 2 * I;
-    const uint4 g4 = __ldg(reinterpret_cast<const uint4*>(G + grow + c));
-    const uint4 u4 = __ldg(reinterpret_cast<const uint4*>(G + grow + I + c));
-    const uint4 d4 = __ldg(reinterpret_cast<const uint4*>(dh + static_cast<size_t>(n) * I + c));
-    const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g4);
-    const __nv_bfloat162* u2 = reinterpret_cast<const __nv_bfloat162*>(&u4);
-    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&d4);
-    uint4 og, ou;
-    __nv_bfloat162* og2 = reinterpret_cast<__nv_bfloat162*>(&og);
-    __nv_bfloat162* ou2 = reinterpret_cast<__nv_bfloat162*>(&ou);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float2 g = __bfloat1622float2(g2[i]), u = __bfloat1622float2(u2[i]);
-      const float2 d = __bfloat1622float2(d2[i]);
-      const float sx = 1.0f / (1.0f + expf(-g.x)), sy = 1.0f / (1.0f + expf(-g.y));
-      og2[i] = __floats2bfloat162_rn(d.x * u.x * sx * (1.0f + g.x * (1.0f - sx)),
-                                     d.y * u.y * sy * (1.0f + g.y * (1.0f - sy)));
-      ou2[i] = __floats2bfloat162_rn(d.x * g.x * sx, d.y * g.y * sy);
-    }
-    *reinterpret_cast<uint4*>(dG + grow + c) = og;
-    *reinterpret_cast<uint4*>(dG + grow + I + c) = ou;
-  }
-}
-
 __global__ void fill_kernel(float* __restrict__ p, size_t n, float v) {
   for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<size_t>(gridDim.x) * blockDim.x)
@@ -233,18 +199,6 @@ cudaError_t launch_gate_backward(const float* logits, const int32_t* topk_idx,
   count_launch();
   gate_backward_kernel<<<warp_grid(T), 256, 0, s>>>(logits, topk_idx, dgates, T, E, k, sigmoid,
                                                     renorm, scale, dlogits);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_swiglu_backward(const void* G, const void* dh, int S, int I, void* dG,
-                                   cudaStream_t s) {
-  const long items = static_cast<long>(S) * (I / 8);
-  const long blocks = (items + 255) / 256;
-  const long cap = static_cast<long>(num_sms()) * 8;
-  count_launch();
-  swiglu_backward_kernel<<<static_cast<unsigned>(blocks < cap ? blocks : cap), 256, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(G), static_cast<const __nv_bfloat16*>(dh), S, I,
-      static_cast<__nv_bfloat16*>(dG));
   return cudaGetLastError();
 }
 

@@ -61,7 +61,8 @@ namespace {
 
 using namespace gemm;
 
-template <int kCta, int kTm, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3>
+template <int kCta, int kTm, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3,
+          bool kDGate>
 __global__ void __launch_bounds__(kThreads, 1)
 grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const TcParams p) {
@@ -75,7 +76,7 @@ grouped_gemm_tc(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
   if constexpr (kCta == 2) cluster_sync();  // the peer's barriers exist before anyone signals them
   tc_fence_after();
   Pipe pipe;
-  gemm_phase<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm>(&tmA, &tmB, p, sm, pipe);
+  gemm_phase<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, kDGate>(&tmA, &tmB, p, sm, pipe);
   tc_fence_before();
   __syncthreads();
   // in a pair, neither CTA leaves while the other may still touch its shared memory
@@ -114,7 +115,7 @@ grouped_gemm_promote(const __grid_constant__ CUtensorMap tmA,
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
-template <int kCta, int kTm, bool kBS, int kBFmt, bool kSw, bool kE4>
+template <int kCta, int kTm, bool kBS, int kBFmt, bool kSw, bool kE4, bool kDG = false>
 cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   const int K = linear1 ? a.H : a.I;
   const int w_rows = linear1 ? 2 * a.I : a.H;
@@ -138,8 +139,9 @@ cudaError_t launch_tc(const FfnArgs& a, bool linear1, cudaStream_t s) {
   p.b_scales = a.w_scales;
   p.out = a.out;
   p.out_scales = a.out_scales;
+  p.dh = a.dh;
   p.err = a.err;
-  auto kern = grouped_gemm_tc<kCta, kTm, kBS, kBFmt, kSw, kE4>;
+  auto kern = grouped_gemm_tc<kCta, kTm, kBS, kBFmt, kSw, kE4, kDG>;
   const size_t smem = Cfg<kCta, kTm>::kSmem;
   cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
@@ -195,12 +197,12 @@ cudaError_t launch_promote(const FfnArgs& a, bool linear1, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <bool kBS, int kBFmt, bool kSw, bool kE4>
+template <bool kBS, int kBFmt, bool kSw, bool kE4, bool kDG = false>
 cudaError_t launch_tc_any(const FfnArgs& a, bool linear1, cudaStream_t s) {
   switch (gemm_tile_shape(a.act, a.S, a.E, true)) {
-    case 2: return launch_tc<2, kBM, kBS, kBFmt, kSw, kE4>(a, linear1, s);
-    case 3: return launch_tc<1, 32, kBS, kBFmt, kSw, kE4>(a, linear1, s);
-    default: return launch_tc<1, kBM, kBS, kBFmt, kSw, kE4>(a, linear1, s);
+    case 2: return launch_tc<2, kBM, kBS, kBFmt, kSw, kE4, kDG>(a, linear1, s);
+    case 3: return launch_tc<1, 32, kBS, kBFmt, kSw, kE4, kDG>(a, linear1, s);
+    default: return launch_tc<1, kBM, kBS, kBFmt, kSw, kE4, kDG>(a, linear1, s);
   }
 }
 
@@ -234,6 +236,12 @@ cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s) {
   if (a.act == MOE_E4M3 && a.wt == MOE_E4M3) return launch_tc_any<true, 0, true, true>(a, true, s);
   if (a.act == MOE_E4M3 && a.wt == MOE_E2M1) return launch_tc_any<true, 5, true, true>(a, true, s);
   return cudaErrorNotSupported;
+}
+
+cudaError_t launch_linear1_dgate_tc(const FfnArgs& a, cudaStream_t s) {
+  if (a.E > kMaxE) return cudaErrorNotSupported;
+  if (a.act != MOE_BF16 || a.wt != MOE_BF16 || a.dh == nullptr) return cudaErrorNotSupported;
+  return launch_tc_any<false, 0, true, false, true>(a, true, s);
 }
 
 cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s) {

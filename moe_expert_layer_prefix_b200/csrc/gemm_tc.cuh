@@ -102,6 +102,7 @@ struct TcParams {
   const void* b_scales;    // E4M3: fp32 [E, w_rows/128, K/128]; E2M1: u8 [E, w_rows, K/32]
   void* out;
   float* out_scales;       // linear-1 with E4M3 h
+  const void* dh;          // linear-1 backward form (kDGate): the gradient of h, BF16 [S, I]
   int* err;
 };
 
@@ -353,9 +354,11 @@ __device__ __forceinline__ void gemm_fini(const Smem& sm) {
 // kind::mxf8f6f4 with A = E4M3 and B = E4M3 (kBFmt 0) or E2M1 (kBFmt 5).  kSwiGLU: linear-1
 // epilogue, else linear-2.  kOutE4M3: linear-1 stores h as E4M3 + 1x128 scales (else BF16).
 // kStager: the MMA issuer polls the stager warp's ready count instead of waiting on the
-// stage barriers itself (E2M1 weights only; gemm_phase picks it).
+// stage barriers itself (E2M1 weights only; gemm_phase picks it).  kDGate (with kSwiGLU,
+// BF16): the backward form of linear-1, whose epilogue turns the recomputed pre-activations
+// (g, u) and the gradient of h into the gradient of both (dg, du) instead of storing h.
 template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm,
-          bool kStager>
+          bool kStager, bool kDGate = false>
 __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
                                              const TcParams& p, const Smem& sm, Pipe& pipe) {
   using C = Cfg<kCta, kTm>;
@@ -939,7 +942,44 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
         if constexpr (kPair) mbar_arrive_cluster(acc_empty_lead);
         else mbar_arrive(&ss.acc_empty);
       }
-      if constexpr (kSwiGLU) {
+      if constexpr (kSwiGLU && kDGate) {
+        // h = silu(g) u: dg = dh u silu'(g) = dh u s (1 + g (1 - s)), du = dh silu(g) = dh g s
+        // with s = sigmoid(g), on the fp32 accumulator; the row's 64 columns of dh come in
+        // (16-byte loads), its 64 gate and 64 up columns of dG [S, 2I] go out
+        if (valid) {
+          const int col0 = tile.nb * 128 + 64 * half;
+          const uint4* dhp = reinterpret_cast<const uint4*>(
+              static_cast<const __nv_bfloat16*>(p.dh) + static_cast<size_t>(row) * p.n_out + col0);
+          __nv_bfloat16* dg_row = static_cast<__nv_bfloat16*>(p.out) +
+                                  static_cast<size_t>(row) * 2 * p.n_out + col0;
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 dv = __ldg(dhp + v);
+            const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+            uint32_t wg[4], wu[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 dd = __bfloat1622float2(d2[i]);
+              float rg[2], ru[2];
+#pragma unroll
+              for (int c = 0; c < 2; ++c) {
+                const float g = __uint_as_float(d[8 * v + 2 * i + c]);
+                const float u = __uint_as_float(d[64 + 8 * v + 2 * i + c]);
+                const float dhv = c == 0 ? dd.x : dd.y;
+                const float sg = 1.0f / (1.0f + expf(-g));
+                rg[c] = dhv * u * sg * (1.0f + g * (1.0f - sg));
+                ru[c] = dhv * g * sg;
+              }
+              const __nv_bfloat162 bg = __floats2bfloat162_rn(rg[0], rg[1]);
+              const __nv_bfloat162 bu = __floats2bfloat162_rn(ru[0], ru[1]);
+              wg[i] = *reinterpret_cast<const uint32_t*>(&bg);
+              wu[i] = *reinterpret_cast<const uint32_t*>(&bu);
+            }
+            reinterpret_cast<uint4*>(dg_row)[v] = make_uint4(wg[0], wg[1], wg[2], wg[3]);
+            reinterpret_cast<uint4*>(dg_row + p.n_out)[v] = make_uint4(wu[0], wu[1], wu[2], wu[3]);
+          }
+        }
+      } else if constexpr (kSwiGLU) {
         float h[64];
 #pragma unroll
         for (int i = 0; i < 64; ++i)
@@ -1030,18 +1070,20 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
 // off that thread is measured faster.  E4M3 and BF16 kinds issue far fewer copies, and
 // shorter K loops do not amortise the hand-off: both lose more to it than they gain.  The
 // choice is per phase; the pipeline counters stay in step across phases of either kind.
-template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm = kBM>
+template <int kCta, bool kBlockScaled, int kBFmt, bool kSwiGLU, bool kOutE4M3, int kTm = kBM,
+          bool kDGate = false>
 __device__ __forceinline__ void gemm_phase(const CUtensorMap* tmA_, const CUtensorMap* tmB_,
                                            const TcParams& p, const Smem& sm, Pipe& pipe) {
+  static_assert(!kDGate || (kSwiGLU && !kBlockScaled), "the backward form: BF16 linear-1");
   if constexpr (kBlockScaled && kBFmt == 5) {
     if (p.K >= 8 * 128) {
-      gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, true>(tmA_, tmB_, p, sm,
-                                                                             pipe);
+      gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, true, kDGate>(
+          tmA_, tmB_, p, sm, pipe);
       return;
     }
   }
-  gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, false>(tmA_, tmB_, p, sm,
-                                                                          pipe);
+  gemm_phase_k<kCta, kBlockScaled, kBFmt, kSwiGLU, kOutE4M3, kTm, false, kDGate>(
+      tmA_, tmB_, p, sm, pipe);
 }
 
 }  // namespace gemm

@@ -43,8 +43,6 @@ cudaError_t launch_combine_backward(const void* dout, const void* y, const int32
 cudaError_t launch_gate_backward(const float* logits, const int32_t* topk_idx,
                                  const float* dgates, int T, int E, int k, int sigmoid,
                                  int renorm, float scale, float* dlogits, cudaStream_t s);
-cudaError_t launch_swiglu_backward(const void* G, const void* dh, int S, int I, void* dG,
-                                   cudaStream_t s);
 // Weight gradients on tensor cores (wgrad_tc.cu): pk = expert-padded segment starts, the
 // slot-major operands transposed into [C, wgrad_pad_cols(S, E)] copies, then the GEMM.
 size_t wgrad_pad_cols(int S, int E);
@@ -68,6 +66,7 @@ struct FfnArgs {
   float* out_scales;           // h_scales (linear-1, E4M3) or null
   int* err;                    // device error word
   int scale_fmt = MOE_SCALE_POW2;  // moe_scale_fmt of the fp32 block scales
+  const void* dh = nullptr;    // launch_linear1_dgate_tc: the gradient of h, BF16 [S, I]
 };
 
 cudaError_t launch_linear1_simt(const FfnArgs& a, cudaStream_t s);
@@ -75,6 +74,10 @@ cudaError_t launch_linear2_simt(const FfnArgs& a, cudaStream_t s);
 
 // tcgen05 path; returns cudaErrorNotSupported for dtype pairs it does not cover.
 cudaError_t launch_linear1_tc(const FfnArgs& a, cudaStream_t s);
+// The backward form of linear-1 (BF16): recomputes the pre-activations g, u = x . W1^T of
+// each slot on the tensor cores and writes out = dG [S, 2I] (dg in columns [0, I), du in
+// [I, 2I)) from them and a.dh, the gradient of h = silu(g) u, without storing g or u.
+cudaError_t launch_linear1_dgate_tc(const FfnArgs& a, cudaStream_t s);
 cudaError_t launch_linear2_tc(const FfnArgs& a, cudaStream_t s);
 
 // 2-D K-major tensor map: rows x K, box {128-byte K slice, 128 rows}, 128-byte swizzle.

@@ -204,7 +204,7 @@ def layer_backward(L: Layer, dout, n_group: int = 1, topk_group: int = 0, scale:
                            n_group, topk_group, scale)
 
 
-def layer_backward_stored(L: Layer, dout, store=None):
+def layer_backward_stored(L: Layer, dout, store=None, return_slots=False):
     """The backward of a BF16 layer with every intermediate stored where the CUDA path stores
     it (`store` rounds a value to its storage format; default BF16 round-to-nearest-even):
 
@@ -212,15 +212,18 @@ def layer_backward_stored(L: Layer, dout, store=None):
         h = store(silu(g) * u),  y = store(h W2^T),  gates w as fp32
       dgates[t, j] = dout[t] . y[slot(t, j)]         (an fp32 result: kept exact here)
       dy_w[slot]   = store(w[t, j] * dout[t])
-      G            = store(x W1^T)                    (pre-activations, recomputed)
       dh           = store(dy_w W2)
-      dG           = store(swiglu_grad(G, dh))        (gate and up halves)
+      dG           = store(swiglu_grad(g, u, dh))     (gate and up halves; the
+                                                       pre-activations g, u = x W1^T
+                                                       are recomputed, not stored)
       dx_slot      = store(dG W1),   dx[t] = store(sum over the token's slots of dx_slot)
       dW1_e = dG_e^T x_e,  dW2_e = dy_w,e^T h_e        (fp32 results: exact here)
       dlogits      = gate_grad(dgates)                (an fp32 result)
 
     With store = identity this is layer_backward up to the fp32 storage of the gates.
-    Returns the same dict as layer_backward."""
+    Returns the same dict as layer_backward; with return_slots, also "slots": the stored
+    per-slot values the weight gradients sum (dG, x, dy_w, h) and dh, rows in dispatch
+    order."""
     from .formats import round_bf16
     st = round_bf16 if store is None else store
     dout = np.asarray(dout, np.float64)
@@ -232,6 +235,7 @@ def layer_backward_stored(L: Layer, dout, store=None):
     xh = L.x_hat()
     T, H = xh.shape
     dx_slot = np.zeros((tok.size, H), np.float64)
+    slots = {}
     dgates = np.zeros_like(w)
     dw1 = dw2 = None
     for e in range(L.E):
@@ -242,7 +246,6 @@ def layer_backward_stored(L: Layer, dout, store=None):
             dw2 = np.zeros((L.E,) + w2.shape, np.float64)
         if a == b:
             continue
-        I = w1.shape[0] // 2
         t, j = tok[a:b], rank[a:b]
         x = xh[t]
         _, gate, up, _ = expert_ffn_exact(x, w1, w2)
@@ -250,16 +253,21 @@ def layer_backward_stored(L: Layer, dout, store=None):
         y = st(h @ w2.T)
         dgates[t, j] = np.einsum("nh,nh->n", dout[t], y)
         dyw = st(w32[t, j][:, None] * dout[t])
-        G = st(x @ w1.T)
         dh = st(dyw @ w2)
-        dg, du = swiglu_grad(G[:, :I], G[:, I:], dh)
+        dg, du = swiglu_grad(gate, up, dh)
         dG = np.concatenate([st(dg), st(du)], axis=1)
         dx_slot[a:b] = st(dG @ w1)
         dw1[e] = dG.T @ x
         dw2[e] = dyw.T @ h
+        if return_slots:
+            for n, v in (("dG", dG), ("x", x), ("dy_w", dyw), ("h", h), ("dh", dh)):
+                slots.setdefault(n, np.zeros((tok.size, v.shape[1]), np.float64))[a:b] = v
     dx = np.zeros((T, H), np.float64)
     np.add.at(dx, tok, dx_slot)
     dl = gate_grad(L.logits, idx, dgates, L.score, L.renorm)
     dbias = None if L.bias is None else np.zeros(L.E, np.float64)
-    return dict(dx=st(dx), dw1=dw1, dw2=dw2, dlogits=dl, dbias=dbias, topk_idx=idx,
-                offsets=offsets)
+    res = dict(dx=st(dx), dw1=dw1, dw2=dw2, dlogits=dl, dbias=dbias, topk_idx=idx,
+               offsets=offsets)
+    if return_slots:
+        res["slots"] = slots
+    return res
