@@ -493,7 +493,7 @@ __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
 
 __device__ __forceinline__ bool grid_sync(uint32_t* bar, int* err, uint32_t expected) {
   __syncthreads();
-  int ok = 1;  // thread 0's verdict, shared through the closing barrier (no shared memory)
+  int ok = 1;  // thread 0's result, shared through the closing barrier (no shared memory)
   if (threadIdx.x == 0) {
     const uint32_t gen = ld_acquire_gpu(bar + 1);
     __threadfence();
