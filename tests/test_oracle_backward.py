@@ -212,3 +212,28 @@ def test_stored_backward_is_close_to_the_exact_backward():
     for n in ("dx", "dw1", "dw2", "dlogits"):
         rel = np.sqrt(np.sum((a[n] - b[n]) ** 2) / np.sum(b[n] ** 2))
         assert 0 < rel < 1e-2, (n, rel)
+
+
+def test_stored_backward_slots_are_what_the_weight_gradients_sum():
+    """The per-slot values the stored backward returns for the GPU tests' rounding allowance
+    are the ones its weight gradients were summed from: dW1_e = dG_e^T x_e and
+    dW2_e = dy_w,e^T h_e over each expert's rows, every value on the BF16 grid, and dG
+    carrying the SwiGLU backward of dh (both halves zero where dh is zero)."""
+    L, dout = _bf16_layer(6, E=5)
+    r = B.layer_backward_stored(L, dout, return_slots=True)
+    s, offs = r["slots"], r["offsets"]
+    assert set(s) == {"dG", "x", "dy_w", "h", "dh"}
+    for n, v in s.items():
+        assert np.array_equal(oracle.round_bf16(v), v), n
+    I = s["h"].shape[1]
+    for e in range(L.E):
+        a, b = int(offs[e]), int(offs[e + 1])
+        assert np.allclose(s["dG"][a:b].T @ s["x"][a:b], r["dw1"][e], rtol=0, atol=1e-9)
+        assert np.allclose(s["dy_w"][a:b].T @ s["h"][a:b], r["dw2"][e], rtol=0, atol=1e-9)
+    zero = s["dh"] == 0
+    assert np.all(s["dG"][:, :I][zero] == 0) and np.all(s["dG"][:, I:][zero] == 0)
+    # without return_slots the result is the same, minus the slots
+    r0 = B.layer_backward_stored(L, dout)
+    assert "slots" not in r0
+    for n in ("dx", "dw1", "dw2", "dlogits"):
+        assert np.array_equal(r0[n], r[n]), n
