@@ -102,7 +102,7 @@ __device__ __forceinline__ void pgemm_phase(const CUtensorMap* tmA_, const CUten
       for (int u = cid; u < units && !*abort; u += ncl) {
         for (int sub = 0; sub < kUnit && !*abort; ++sub) {
           const int t = u * kUnit + sub;
-          const Tile tile = decode_tile(ss, p.E, p.n_tiles, kBM, t);
+          const Tile tile = decode_tile(ss, p.E, p.n_tiles, kBM, t, true);
           const int ebase = tile.e * p.w_rows;
           for (int kb = 0; kb < KB; ++kb) {
             const int stage = static_cast<int>(it % kPStages);
@@ -196,7 +196,7 @@ __device__ __forceinline__ void pgemm_phase(const CUtensorMap* tmA_, const CUten
       float hkeep[32];  // linear-1: the first tile's h values of this thread (E4M3 output)
       for (int sub = 0; sub < kUnit && ok; ++sub) {
         const int t = u * kUnit + sub;
-        const Tile tile = decode_tile(ss, p.E, p.n_tiles, kBM, t);
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, kBM, t, true);
         const int row0 = tile.m0 + q * 32;
         const int row = row0 + lane;
         const bool valid = row < tile.m_end;

@@ -152,18 +152,34 @@ struct Tile {
   int e, m0, m_end, nb;
 };
 
+// Tile t of the list: expert e owns tiles [mb_start[e], mb_start[e + 1]) x n_tiles, numbered
+// n-block-major inside the expert (all of its m-blocks for n-block 0, then n-block 1, ...),
+// so that the CTAs working side by side on an expert with several m-blocks share each weight
+// tile while it is in L2 instead of reading it again a wave later.  mb_major numbers them
+// m-block-major instead (consecutive tiles: the n-blocks of one m-block).
 __device__ __forceinline__ Tile decode_tile(const SharedState& ss, int E, int n_tiles, int tile_m,
-                                            int t) {
-  const int mb = t / n_tiles;
-  Tile tile;
-  tile.nb = t - mb * n_tiles;
-  int lo = 0, hi = E;  // mb_start[lo] <= mb < mb_start[hi]
+                                            int t, bool mb_major = false) {
+  const int q = t / n_tiles;  // in [mb_start[e], mb_start[e + 1]) exactly for e's tiles
+  int lo = 0, hi = E;  // mb_start[lo] <= q < mb_start[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (ss.mb_start[mid] <= mb) lo = mid; else hi = mid;
+    if (ss.mb_start[mid] <= q) lo = mid; else hi = mid;
   }
+  Tile tile;
   tile.e = lo;
-  tile.m0 = ss.offs[lo] + (mb - ss.mb_start[lo]) * tile_m;
+  int mb;  // the m-block inside the expert
+  if (mb_major) {
+    // (no second division: this sits on the issuing threads' path once per tile, and the
+    // tiles of short K loops are only a few k-steps long)
+    mb = q - ss.mb_start[lo];
+    tile.nb = t - q * n_tiles;
+  } else {
+    const int nmb = ss.mb_start[lo + 1] - ss.mb_start[lo];
+    const int local = t - ss.mb_start[lo] * n_tiles;
+    tile.nb = local / nmb;
+    mb = local - tile.nb * nmb;
+  }
+  tile.m0 = ss.offs[lo] + mb * tile_m;
   tile.m_end = ss.offs[lo + 1];
   return tile;
 }
@@ -377,6 +393,11 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
   constexpr int kElemsPerRow = kBlockScaled ? 128 : 64;  // K elements per stage
   const int KB = p.K / kElemsPerRow;
   static_assert(!kStager || kBlockScaled, "the stager converts block scales");
+  // tile order (every role decodes the same list): n-block-major inside an expert, so that
+  // side-by-side CTAs share a weight tile, where a k-step's weight tile is the larger operand
+  // (E4M3, BF16: 256 rows x 128 bytes against 128 x 128); for E2M1 weights the two are equal
+  // and m-block-major, where they share the activation tile, measured faster
+  constexpr bool kMbMajor = kBlockScaled && kBFmt == 5;
   const uint32_t tmem = ss.tmem_base;
   const int total = ss.mb_total * p.n_tiles;
   volatile int* abort = &ss.abort;
@@ -389,7 +410,7 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
       uint32_t it = pipe.prod_it;
       const uint32_t it0 = it;
       for (int t = cid; t < total && !*abort; t += ncl) {
-        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t, kMbMajor);
         const int arow = tile.m0 + static_cast<int>(rank) * kTm;
         // B rows of this CTA: linear-1 gate rows [nb*128, +128) then up rows [I + nb*128, +128);
         // linear-2 rows [nb*256, +256); a pair splits them between its two CTAs
@@ -588,7 +609,7 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
       uint32_t gi = g0;
       bool ok = true;
       for (int lt = cid; lt < total && ok; lt += ncl) {
-        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt, kMbMajor);
         // only the tile's own rows are staged: the MMA's other rows (past the expert's end,
         // or past a small tile's 32) are never stored, and their scales may not exist yet
         uint32_t arow_ok = 0;
@@ -692,7 +713,7 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
     for (int lt = cid; lt < total && ok; lt += ncl) {
       uint32_t arow_ok = 0;  // rows of this tile this lane converts (as the loader staged them)
       if constexpr (kBlockScaled) {
-        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt);
+        const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, lt, kMbMajor);
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           const int m = tile.m0 + static_cast<int>(rank) * kBM + lane + 32 * c;
@@ -820,7 +841,8 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
         const uint32_t gi = g0 + static_cast<uint32_t>(i);
         const int slot = static_cast<int>(gi % kSfGroups);
         if (i % NG == 0) {
-          const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, cid + (i / NG) * ncl);
+          const Tile tile =
+              decode_tile(ss, p.E, p.n_tiles, C::kTileM, cid + (i / NG) * ncl, kMbMajor);
           arow_ok = 0;
 #pragma unroll
           for (int c = 0; c < 4; ++c) {
@@ -908,7 +930,7 @@ __device__ __forceinline__ void gemm_phase_k(const CUtensorMap* tmA_, const CUte
     const uint32_t acc_empty_lead = mapa_shared(smem_u32(&ss.acc_empty), 0);
     for (int t = cid; t < total && !*abort; t += ncl) {
       const uint32_t acc_phase = tiles & 1u;
-      const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t);
+      const Tile tile = decode_tile(ss, p.E, p.n_tiles, C::kTileM, t, kMbMajor);
       // every lane waits; the decision is made warp-uniform so that the .sync.aligned
       // TMEM loads below always run with the full warp
       const bool ready =
