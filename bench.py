@@ -38,8 +38,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 # smaller case with the same rows per expert (dram__bytes_read.sum + dram__bytes_write.sum
 # of one launch).  Used for the roofline's "traffic".
 TRAFFIC_RATIO = {
-    ("v3_fp8", "linear1"): (1.153, "the V3-shaped layer at T=1024, E=32"),
-    ("v3_fp8", "linear2"): (0.972, "the V3-shaped layer at T=1024, E=32"),
+    ("v3_fp8", "linear1"): (1.022, "the V3-shaped layer at T=1024, E=32"),
+    ("v3_fp8", "linear2"): (0.964, "the V3-shaped layer at T=1024, E=32"),
     ("decode_fp8_fp4", "linear1"): (1.013, "the decode-shaped layer at E=64"),
 }
 
