@@ -219,10 +219,13 @@ moe_status moe_combine(const void* y, int y_dt, const int32_t* slot_of, const fl
 /* The whole layer: route -> dispatch -> linear-1 + SwiGLU -> linear-2 -> combine, all
  * intermediates in the workspace (moe_workspace_size(MOE_OP_FORWARD, ...) bytes).
  * (jiqizhixin, section "Mega MoE 是什么？", the mega-kernel paragraph.)
- * For the tensor-core formats (BF16, E4M3 activations) this is ONE persistent cooperative
- * kernel launch (plus an 8-byte memset of its grid barrier) running every step in phases;
- * it produces the same bytes as the chain moe_route, moe_dispatch, moe_expert_linear1,
- * moe_expert_linear2, moe_combine.  The fp32 layer runs that chain.
+ * For the tensor-core formats (BF16, E4M3 activations with power-of-two block scales) this
+ * is ONE persistent cooperative kernel launch (plus an 8-byte memset of its grid barrier)
+ * running every step in phases, with the expert GEMMs' tile shape the chain would use (for
+ * 256-row CTA-pair tiles it is a cluster launch of as many pairs as can be resident at
+ * once); it produces the same bytes as the chain moe_route, moe_dispatch,
+ * moe_expert_linear1, moe_expert_linear2, moe_combine.  The fp32 layer and weights marked
+ * MOE_SCALE_FP32 run that chain.
  * topk_idx / topk_w / expert_offsets may be NULL; when given, the routing result and the
  * per-expert offsets are written there too.
  * x is in format W->act with x_scales for E4M3; for E4M3 layers x_scales may instead be NULL,
