@@ -63,3 +63,24 @@ def test_algorithmic_units_match_the_published_workload_figures():
     weights = (a["linear1"]["bytes"] - mx.S * (mx.H + mx.I) * 2 +
                a["linear2"]["bytes"] - mx.S * mx.I * 2 - mx.S * mx.H * 2)
     assert abs(weights / 1e9 - 2.82) < 0.01, weights
+
+
+def test_algorithmic_bytes_of_the_decode_weights_and_the_router():
+    """The byte counts behind the HBM rooflines, against hand-computed figures: the decode
+    layer's E2M1 weights with their UE8M0 per-32 scales are 3 x I x H x (1/2 + 1/32) bytes
+    per expert (23.4 MB; 5.89 GB for the 252 experts its routing touches), and the router
+    reads T x E fp32 logits and writes T x k indices and gates (69.2 MB on the skewed
+    layer)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    wl = synth.WORKLOADS["decode_fp8_fp4"]
+    per_expert = 3 * wl.I * wl.H * (0.5 + 1 / 32)
+    assert abs(per_expert / 1e6 - 23.4) < 0.05
+    a = bench.algorithmic(wl, 252)
+    act = wl.S * (wl.H + wl.H // 128 * 4) + 2 * wl.S * (wl.I + wl.I // 128 * 4) + wl.S * wl.H * 2
+    weights = a["linear1"]["bytes"] + a["linear2"]["bytes"] - act
+    assert abs(weights / 1e9 - 5.89) < 0.01, weights
+    sk = synth.WORKLOADS["skewed_fp8_fp4"]
+    assert bench.algorithmic(sk, sk.E)["route"]["bytes"] == sk.T * sk.E * 4 + sk.T * sk.k * 8
+    assert abs(bench.algorithmic(sk, sk.E)["route"]["bytes"] / 1e6 - 69.2) < 0.1
