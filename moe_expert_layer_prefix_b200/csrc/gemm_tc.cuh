@@ -8,7 +8,8 @@
 //
 // Both GEMMs have the form  D[m, n] = sum_k A[m, k] * B[n, k]  per expert, A = the expert's
 // rows of x_perm (or h), B = the expert's K-major weight matrix.  Persistent CTAs (one per
-// SM) walk a static list of output tiles (expert, m-block, n-block) of N = 256 columns.
+// SM) walk a static list of output tiles (expert, m-block, n-block) of N = 256 columns
+// (decode_tile gives its order).
 // Tile shapes (Cfg below):
 //   single  one CTA, M = 128: A 128 x 128 B and B 256 x 128 B per k-step, 4 stages
 //   small   one CTA, 32-row m-blocks: a 32-row A box, 5 stages
@@ -38,9 +39,10 @@
 //               columns, so that the accumulator is read out in a quarter of the time and
 //               handed back to the MMA issuer before any arithmetic: SwiGLU + BF16 / E4M3
 //               requantisation (linear-1; the two halves of a row exchange their partial
-//               amax through shared memory) or BF16 conversion (linear-2); 16-byte global
-//               stores, for linear-2 after lane pairs swap chunks so that every store writes
-//               whole 32-byte sectors
+//               amax through shared memory), or in the backward form of linear-1 the
+//               gradients of gate and up from dh, or BF16 conversion (linear-2); 16-byte
+//               global stores, for linear-2 after lane pairs swap chunks so that every store
+//               writes whole 32-byte sectors
 //
 // linear-1 tiles take B rows [n*128, n*128+128) (gate) and [I + n*128, ...) (up), so the
 // accumulator holds gate in columns 0..127 and up in 128..255 and each tile yields 128 h
